@@ -1,0 +1,115 @@
+"""Plant plausible mistakes in the oracle (on the CPU) and check that a pin catches each.
+
+Each mutation replaces one oracle function by a subtly wrong copy; the listed
+pin tests must then fail.  This guards the pins themselves: a pin that still
+passes with a dropped term, a wrong sign or index, or a transposed operand
+would not be pinning anything.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+import oracle.sol_oracle as so
+from tests import test_oracle_pins as pins
+
+
+def _prologue_rope_sign(x, gamma, grid, split, theta, eps):
+    y = np.asarray(x, np.float64)
+    H, D = y.shape[2], y.shape[3]
+    y = y / np.sqrt(np.mean(y * y, axis=-1, keepdims=True) + eps) * np.asarray(gamma).reshape(H, D)
+    phi = so.rope_angles(grid, split, theta)
+    c, s = np.cos(phi)[None, :, None, :], np.sin(phi)[None, :, None, :]
+    out = np.empty_like(y)
+    out[..., 0::2] = y[..., 0::2] * c + y[..., 1::2] * s        # rotates the other way
+    out[..., 1::2] = -y[..., 0::2] * s + y[..., 1::2] * c
+    return out
+
+
+def _angles_axis_reversed(grid, split, theta):
+    T, Hg, Wg = grid
+    n = np.arange(T * Hg * Wg)
+    pos = (n % Wg, (n // Wg) % Hg, n // (Hg * Wg))               # x, y, t instead of t, y, x
+    cols = []
+    for axis in range(3):
+        for i in range(split[axis] // 2):
+            cols.append(pos[axis] * theta ** (-2.0 * i / split[axis]))
+    return np.stack(cols, axis=1)
+
+
+def _prologue_eps_outside(x, gamma, grid, split, theta, eps):
+    y = np.asarray(x, np.float64)
+    H, D = y.shape[2], y.shape[3]
+    y = y / (np.sqrt(np.mean(y * y, axis=-1, keepdims=True)) + eps) * np.asarray(gamma).reshape(H, D)
+    phi = so.rope_angles(grid, split, theta)
+    c, s = np.cos(phi)[None, :, None, :], np.sin(phi)[None, :, None, :]
+    out = np.empty_like(y)
+    out[..., 0::2] = y[..., 0::2] * c - y[..., 1::2] * s
+    out[..., 1::2] = y[..., 0::2] * s + y[..., 1::2] * c
+    return out
+
+
+def _pool_full_block_divisor(x, block):
+    x = np.asarray(x, np.float64)
+    B, N, H, D = x.shape
+    nb = -(-N // block)
+    out = np.empty((B, H, nb, D))
+    for i in range(nb):
+        out[:, :, i, :] = x[:, i * block:(i + 1) * block].sum(axis=1) / block
+    return out
+
+
+
+def _topk_ties_high(scores, k):
+    s = np.asarray(scores, np.float64)
+    n = s.shape[-1]
+    rev = s[..., ::-1]
+    order = np.argsort(-rev, axis=-1, kind="stable")[..., :k]
+    return np.sort(n - 1 - order, axis=-1).astype(np.int32)
+
+
+def _attention_rows_no_scale(q, k, v, idx, block, scale, b, h, i):
+    return so.__dict__["_orig_rows"](q, k, v, idx, block, 1.0, b, h, i)
+
+
+def _attention_rows_lse_no_max(q, k, v, idx, block, scale, b, h, i):
+    o, lse = so.__dict__["_orig_rows"](q, k, v, idx, block, scale, b, h, i)
+    N = q.shape[1]
+    rows = np.arange(i * block, min(N, (i + 1) * block))
+    cols = np.concatenate([np.arange(j * block, min(N, (j + 1) * block)) for j in np.asarray(idx[b, h, i])])
+    logits = scale * (np.asarray(q[b, rows, h], np.float64) @ np.asarray(k[b, cols, h], np.float64).T)
+    mx = logits.max(axis=1)
+    return o, lse - mx
+
+
+MUTATIONS = [
+    ("qk_prologue", _prologue_rope_sign, [pins.test_prologue_hand_case]),
+    ("rope_angles", _angles_axis_reversed, [pins.test_prologue_hand_case]),
+    ("qk_prologue", _prologue_eps_outside, [pins.test_prologue_hand_case, pins.test_prologue_gamma_indexing_and_eps]),
+    ("block_pool", _pool_full_block_divisor, [pins.test_pool_hand_case]),
+    ("topk_blocks", _topk_ties_high, [pins.test_topk_brute_force_with_ties]),
+    ("sparse_attention_rows", _attention_rows_no_scale, [pins.test_attention_all_blocks_equals_dense_library_attention]),
+    ("sparse_attention_rows", _attention_rows_lse_no_max, [pins.test_attention_all_blocks_equals_dense_library_attention,
+                                                           pins.test_attention_hand_cases]),
+]
+
+
+@pytest.mark.parametrize("name,bad,tests", MUTATIONS, ids=[m[1].__name__ for m in MUTATIONS])
+def test_pins_catch_planted_mistake(monkeypatch, name, bad, tests):
+    monkeypatch.setitem(so.__dict__, "_orig_rows", so.sparse_attention_rows)
+    monkeypatch.setattr(so, name, bad)
+    monkeypatch.setattr(oracle, name, bad)
+    for t in tests:
+        with pytest.raises(AssertionError):
+            t()
+
+
+def test_scores_transposition_is_caught(monkeypatch):
+    # A transposed score matrix (s_ji for s_ij) must fail the dense-block closed form.
+    bad = lambda qbar, kbar: np.swapaxes(so.__dict__["_orig_scores"](qbar, kbar), -1, -2)  # noqa: E731
+    monkeypatch.setitem(so.__dict__, "_orig_scores", so.block_scores)
+    monkeypatch.setattr(so, "block_scores", bad)
+    monkeypatch.setattr(oracle, "block_scores", bad)
+    with pytest.raises(AssertionError):
+        pins.test_scores_equal_mean_of_dense_logit_blocks()
