@@ -1,0 +1,361 @@
+"""Benchmark of the Sol-Attn hot path on B200: QK-RMSNorm + 3D RoPE ->
+block select -> block-sparse attention, one pass of the whole chain per step.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 4] [--impl ours|reference]
+
+Prints ONE JSON line (rank 0).  `value` is the selected-FLOP rate of the whole
+chain step (selected attention FLOPs / device time of prologue + select +
+attention), summed over ranks; each rank runs its own independent clip of the
+workload (weak scaling, no collective on the data path).  Inputs stay resident
+in HBM during the device-timed region and are far larger than L2 (no flush
+needed).  `e2e` times the same chain through host buffers: pinned host -> device
+copies of the raw Q, K, V and the device -> host copy of O and LSE are inside
+the timed region.  `--impl reference` times the fp64 CPU oracle on a bounded
+sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import WORKLOADS, make_inputs  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def load_ncu_traffic(kernel: str):
+    """Per-launch DRAM bytes of `kernel` from the committed ncu summary, or None."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        for line in f:
+            if line.startswith("dram_bytes_per_launch:"):
+                return float(line.split(":", 1)[1].split()[0])
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        self.proc = None
+        self.device = device
+
+    def __enter__(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"]
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.device).uuid)
+            cmd += ["-i", uuid if uuid.startswith("GPU-") else "GPU-" + uuid]
+        except Exception:
+            pass
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except FileNotFoundError:
+            self.proc = None
+        time.sleep(0.25)
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            out, _ = self.proc.communicate(timeout=10)
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------- oracle timing
+def oracle_attention_sample(wl, inp, topk, n_units: int, seed: int):
+    """Times the fp64 oracle on n_units (b, h, query block) units of the workload
+    with random valid selections; returns (selected FLOPs, seconds, threads)."""
+    import oracle as orc
+    from workloads import random_index_lists
+    rng = np.random.default_rng([seed, 17])
+    q, k, v = (inp[n].float().numpy() for n in ("q", "k", "v"))
+    idx = random_index_lists(1, 1, wl.nb, topk, seed=seed).numpy()[0, 0]
+    flops = 0
+    t0 = time.perf_counter()
+    for _ in range(n_units):
+        b, h, i = int(rng.integers(0, wl.B)), int(rng.integers(0, wl.H)), int(rng.integers(0, wl.nb))
+        sel = np.zeros((wl.B, wl.H, wl.nb, topk), dtype=np.int32)
+        sel[b, h, i] = idx[i]
+        orc.sparse_attention_rows(q, k, v, sel, wl.block, 1.0 / math.sqrt(wl.D), b, h, i)
+        nq = min(wl.block, wl.N - i * wl.block)
+        nk = sum(min(wl.block, wl.N - j * wl.block) for j in idx[i])
+        flops += 4 * nq * nk * wl.D
+    dt = time.perf_counter() - t0
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max((p.get("num_threads", 1) for p in threadpool_info()), default=1)
+    except Exception:
+        threads = 1
+    return flops, dt, threads
+
+
+def run_reference(args, wl, world, rank):
+    if rank != 0:
+        return
+    topk = wl.topk[0]
+    inp = make_inputs(wl, seed=0, names=("q", "k", "v"))
+    units = args.ref_units
+    for _ in range(args.warmup):
+        oracle_attention_sample(wl, inp, topk, 1, seed=123)
+    tot_f, tot_t, threads = 0, 0.0, 1
+    for s in range(args.steps):
+        f, t, threads = oracle_attention_sample(wl, inp, topk, units, seed=s)
+        tot_f += f
+        tot_t += t
+    value = tot_f / tot_t / 1e12
+    sample = (f"fp64 oracle attention on {units} random (b, h, query block) units per step with k={topk} "
+              f"random kept blocks of workload {wl.config_id}; value = their selected FLOPs / CPU time")
+    line = {
+        "impl": "reference", "metric": "sparse-attn effective TFLOP/s (selected FLOPs)", "value": value,
+        "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": tot_t / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "config_id": wl.config_id, "B": wl.B, "N": wl.N, "H": wl.H, "D": wl.D,
+                   "block": wl.block, "topk": topk, "parallelism": f"independent clip per rank x{world}"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- our arm
+def run_ours(args, wl, world, rank, local):
+    import block_sparse_attention_sol_b200 as sol
+    topk = wl.topk[0]
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    inp = make_inputs(wl, seed=rank)
+    host = {n: inp[n].pin_memory() for n in ("q", "k", "v")}
+    d = {n: inp[n].to(dev) for n in ("q", "k", "v", "gamma_q", "gamma_k")}
+    q = torch.empty_like(d["q"])
+    k = torch.empty_like(d["k"])
+    o = torch.empty_like(d["q"])
+    lse = torch.empty((wl.B, wl.H, wl.N), dtype=torch.float32, device=dev)
+    idx = torch.empty((wl.B, wl.H, wl.nb, topk), dtype=torch.int32, device=dev)
+    shape = sol.SolShape(wl.B, wl.N, wl.H, wl.D, *wl.grid)
+    ws = torch.empty(sol.sol_block_select_workspace_bytes(shape, wl.block), dtype=torch.uint8, device=dev)
+    o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    lse_host = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+
+    def chain(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        sol.sol_qk_prologue(d["q"], d["k"], d["gamma_q"], d["gamma_k"], wl.grid, wl.rope_split, wl.rope_theta,
+                            wl.eps, q_out=q, k_out=k)
+        if ev is not None:
+            ev[1].record(stream)
+        sol.sol_block_select(q, k, wl.grid, wl.block, topk, workspace=ws, idx_out=idx)
+        if ev is not None:
+            ev[2].record(stream)
+        sol.sol_sparse_attn_fwd(q, k, d["v"], idx, wl.grid, wl.block, o=o, lse=lse)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        chain()
+    torch.cuda.synchronize(dev)
+    if sol.sol_check_device_status() != sol.SOL_OK:
+        raise RuntimeError("device-side error during warm-up")
+
+    # device-timed region: inputs resident in HBM
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    with sampler:
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        start.record(stream)
+        for s in range(args.steps):
+            chain(evs[s])
+        stop.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+    status = sol.sol_check_device_status()
+    if status != sol.SOL_OK:
+        raise RuntimeError(f"device-side error in the timed region: {sol.sol_status_string(status)}")
+    ms_local = start.elapsed_time(stop) / args.steps
+    ms = max_over_ranks(ms_local, world)
+    stage_ms = {name: sum(e[i].elapsed_time(e[i + 1]) for e in evs) / args.steps
+                for i, name in enumerate(("prologue", "select", "attention"))}
+
+    # end to end through host buffers
+    e2e_start, e2e_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_steps = args.e2e_steps or args.steps
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    e2e_start.record(stream)
+    for _ in range(e2e_steps):
+        d["q"].copy_(host["q"], non_blocking=True)
+        d["k"].copy_(host["k"], non_blocking=True)
+        d["v"].copy_(host["v"], non_blocking=True)
+        chain()
+        o_host.copy_(o, non_blocking=True)
+        lse_host.copy_(lse, non_blocking=True)
+    e2e_stop.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    e2e_ms = max_over_ranks(e2e_start.elapsed_time(e2e_stop) / e2e_steps, world)
+    h2d = sum(host[n].numel() * host[n].element_size() for n in ("q", "k", "v"))
+    d2h = o_host.numel() * o_host.element_size() + lse_host.numel() * lse_host.element_size()
+
+    flops = wl.selected_flops(topk)          # selected attention FLOPs of one step (one clip)
+    value = flops * world / (ms * 1e-3) / 1e12
+    e2e_value = flops * world / (e2e_ms * 1e-3) / 1e12
+    peaks = load_peaks()
+    att_s = stage_ms["attention"] * 1e-3
+    achieved = flops / att_s / 1e12
+    traffic = load_ncu_traffic("sparse_attn_fwd")
+    io_bytes = wl.B * wl.N * wl.H * wl.D * 2
+    prologue_bytes = 4 * io_bytes
+    select_bytes = 2 * io_bytes + 4 * wl.B * wl.H * wl.nb * topk
+    clocks = sampler.summary()
+    if rank != 0:
+        return
+    line = {
+        "metric": "sparse-attn effective TFLOP/s (selected FLOPs)",
+        "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wl.name, "config_id": wl.config_id, "B": wl.B, "N": wl.N, "H": wl.H, "D": wl.D,
+                   "grid": list(wl.grid), "block": wl.block, "topk": topk,
+                   "selected_tflop_per_step": flops / 1e12,
+                   "parallelism": f"independent clip per rank x{world}",
+                   "l2": f"inputs {5 * io_bytes / 1e9:.1f} GB resident, > {L2_BYTES >> 20} MB L2; no flush"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
+                     "kernel": "sol::attn100::sparse_attn_fwd_kernel",
+                     "peak_source": f"{peaks['source']} bf16 dense (burst)"},
+        "stages": {
+            "prologue": {"ms": stage_ms["prologue"], "GB/s": prologue_bytes / stage_ms["prologue"] / 1e6,
+                         "frac_hbm": prologue_bytes / stage_ms["prologue"] / 1e6 / peaks["hbm_gbs"]},
+            "select": {"ms": stage_ms["select"], "GB/s": select_bytes / stage_ms["select"] / 1e6,
+                       "frac_hbm": select_bytes / stage_ms["select"] / 1e6 / peaks["hbm_gbs"]},
+            "attention": {"ms": stage_ms["attention"], "TFLOP/s": achieved,
+                          "frac_bf16": achieved / peaks["bf16_tflops"]},
+            "hbm_peak_gbs": peaks["hbm_gbs"],
+        },
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e2e_ms},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        f, t, threads = oracle_attention_sample(wl, inp, topk, args.cpu_units, seed=99)
+        line["cpu_baseline"] = {
+            "value": f / t / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": f"fp64 oracle attention on {args.cpu_units} random (b, h, query block) units with "
+                      f"k={topk} random kept blocks ({f / 1e9:.1f} GFLOP, {t:.1f} s)"}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=40)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", type=int, default=4, help="workload id (1-4 bf16)")
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=0)
+    ap.add_argument("--cpu-units", type=int, default=48)
+    ap.add_argument("--ref-units", type=int, default=24)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    wl = WORKLOADS[args.config]
+    if wl.dtype != "bf16":
+        ap.error("the benchmark runs the bf16 workloads 1-4")
+    world, rank, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            run_reference(args, wl, world, rank)
+        else:
+            run_ours(args, wl, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

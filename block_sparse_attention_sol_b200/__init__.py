@@ -1,0 +1,180 @@
+"""Python binding of libsol, the sm_100a Sol-Attn hot path (see include/sol.h).
+
+Argument marshalling only: every step runs in the CUDA kernels of libsol.so.
+PyTorch provides device memory and the current stream.  There is no fallback:
+if the library is missing this import fails, and every call checks that its
+tensors live on a CUDA device.
+
+Functions (same names as the C ABI):
+    sol_qk_prologue(q_raw, k_raw, gamma_q, gamma_k, grid, ...)  -> (q, k)
+    sol_block_select(q, k, grid, block, topk, ...)              -> idx [, scores]
+    sol_sparse_attn_fwd(q, k, v, idx, grid, block, ...)         -> (o, lse)
+    sol_check_device_status(stream=None)
+    sol_selftest_wait_timeout(limit_us, stream=None)
+    sol_block_select_workspace_bytes(shape, block)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "SolError", "SolShape", "LIB_PATH", "lib",
+    "sol_qk_prologue", "sol_block_select", "sol_block_select_workspace_bytes", "sol_sparse_attn_fwd",
+    "sol_check_device_status", "sol_selftest_wait_timeout", "sol_status_string", "sol_attention_chain",
+    "SOL_OK", "SOL_ERR_INVALID_ARG", "SOL_ERR_UNSUPPORTED", "SOL_ERR_CUDA", "SOL_ERR_TIMEOUT",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsol.so")
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m block_sparse_attention_sol_b200.build` "
+        "(there is no non-CUDA fallback)")
+lib = ctypes.CDLL(LIB_PATH)
+
+SOL_OK, SOL_ERR_INVALID_ARG, SOL_ERR_UNSUPPORTED, SOL_ERR_CUDA, SOL_ERR_TIMEOUT = range(5)
+SOL_F32, SOL_BF16 = 0, 1
+
+
+class SolShape(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in ("B", "N", "H", "D", "grid_t", "grid_h", "grid_w")]
+
+
+class SolError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {sol_status_string(status)}")
+
+
+_P, _I, _F, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+lib.sol_status_string.restype = ctypes.c_char_p
+lib.sol_status_string.argtypes = [_I]
+lib.sol_qk_prologue.restype = _I
+lib.sol_qk_prologue.argtypes = [_P, _P, _P, _P, _P, _P, SolShape, _I, _I, _I, _F, _F, _I, _P]
+lib.sol_block_select_workspace_bytes.restype = _SZ
+lib.sol_block_select_workspace_bytes.argtypes = [SolShape, _I]
+lib.sol_block_select.restype = _I
+lib.sol_block_select.argtypes = [_P, _P, SolShape, _I, _I, _I, _P, _P, _P, _SZ, _P]
+lib.sol_sparse_attn_fwd.restype = _I
+lib.sol_sparse_attn_fwd.argtypes = [_P, _P, _P, _P, SolShape, _I, _I, _F, _I, _P, _P, _P]
+lib.sol_check_device_status.restype = _I
+lib.sol_check_device_status.argtypes = [_P]
+lib.sol_selftest_wait_timeout.restype = _I
+lib.sol_selftest_wait_timeout.argtypes = [ctypes.c_uint, _P]
+
+
+def sol_status_string(status: int) -> str:
+    return lib.sol_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str) -> None:
+    if status != SOL_OK:
+        raise SolError(status, what)
+
+
+def _stream_handle(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return SOL_BF16
+    if t.dtype == torch.float32:
+        return SOL_F32
+    raise TypeError(f"unsupported dtype {t.dtype} (bf16 or fp32)")
+
+
+def _cuda(t: torch.Tensor, name: str) -> torch.Tensor:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def _shape(x: torch.Tensor, grid) -> SolShape:
+    if x.dim() != 4:
+        raise ValueError("activations are [B, N, H, D]")
+    B, N, H, D = x.shape
+    return SolShape(B, N, H, D, int(grid[0]), int(grid[1]), int(grid[2]))
+
+
+def sol_qk_prologue(q_raw, k_raw, gamma_q, gamma_k, grid, rope_split=None, rope_theta=10000.0, eps=1e-6,
+                    q_out=None, k_out=None, stream=None):
+    """Fused QK-RMSNorm + 3D RoPE.  Returns (q, k) with q_raw's shape and dtype."""
+    _cuda(q_raw, "q_raw"), _cuda(k_raw, "k_raw"), _cuda(gamma_q, "gamma_q"), _cuda(gamma_k, "gamma_k")
+    s = _shape(q_raw, grid)
+    if rope_split is None:
+        dh = 2 * (s.D // 6)
+        rope_split = (s.D - 2 * dh, dh, dh)
+    q_out = torch.empty_like(q_raw) if q_out is None else _cuda(q_out, "q_out")
+    k_out = torch.empty_like(k_raw) if k_out is None else _cuda(k_out, "k_out")
+    st = lib.sol_qk_prologue(q_raw.data_ptr(), k_raw.data_ptr(), q_out.data_ptr(), k_out.data_ptr(),
+                             gamma_q.data_ptr(), gamma_k.data_ptr(), s, int(rope_split[0]), int(rope_split[1]),
+                             int(rope_split[2]), float(rope_theta), float(eps), _dtype_code(q_raw),
+                             _stream_handle(stream))
+    _check(st, "sol_qk_prologue")
+    return q_out, k_out
+
+
+def sol_block_select_workspace_bytes(shape: SolShape, block: int) -> int:
+    return int(lib.sol_block_select_workspace_bytes(shape, int(block)))
+
+
+def sol_block_select(q, k, grid, block, topk, workspace=None, idx_out=None, return_scores=False, stream=None):
+    """Block mean-pool + pooled dot-product scores + top-k.  Returns idx int32
+    [B, H, nb, topk] (and the fp32 score matrix when return_scores)."""
+    _cuda(q, "q"), _cuda(k, "k")
+    s = _shape(q, grid)
+    nb = -(-s.N // block)
+    need = sol_block_select_workspace_bytes(s, block)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _cuda(workspace, "workspace")
+    if idx_out is None:
+        idx_out = torch.empty((s.B, s.H, nb, topk), dtype=torch.int32, device=q.device)
+    scores = torch.empty((s.B, s.H, nb, nb), dtype=torch.float32, device=q.device) if return_scores else None
+    st = lib.sol_block_select(q.data_ptr(), k.data_ptr(), s, int(block), int(topk), _dtype_code(q),
+                              _cuda(idx_out, "idx_out").data_ptr(), scores.data_ptr() if scores is not None else None,
+                              workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                              _stream_handle(stream))
+    _check(st, "sol_block_select")
+    return (idx_out, scores) if return_scores else idx_out
+
+
+def sol_sparse_attn_fwd(q, k, v, idx, grid, block, softmax_scale=0.0, o=None, lse=None, stream=None):
+    """Exact softmax attention over the kept blocks.  Returns (o, lse)."""
+    _cuda(q, "q"), _cuda(k, "k"), _cuda(v, "v"), _cuda(idx, "idx")
+    if idx.dtype != torch.int32:
+        raise TypeError("idx must be int32")
+    s = _shape(q, grid)
+    topk = idx.shape[-1]
+    o = torch.empty_like(q) if o is None else _cuda(o, "o")
+    lse = torch.empty((s.B, s.H, s.N), dtype=torch.float32, device=q.device) if lse is None else _cuda(lse, "lse")
+    st = lib.sol_sparse_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), idx.data_ptr(), s, int(block), int(topk),
+                                 float(softmax_scale), _dtype_code(q), o.data_ptr(), lse.data_ptr(),
+                                 _stream_handle(stream))
+    _check(st, "sol_sparse_attn_fwd")
+    return o, lse
+
+
+def sol_check_device_status(stream=None) -> int:
+    """Synchronises the stream; returns the library status code (SOL_OK, SOL_ERR_TIMEOUT, ...)."""
+    return int(lib.sol_check_device_status(_stream_handle(stream)))
+
+
+def sol_selftest_wait_timeout(limit_us: int, stream=None) -> None:
+    _check(lib.sol_selftest_wait_timeout(int(limit_us), _stream_handle(stream)), "sol_selftest_wait_timeout")
+
+
+def sol_attention_chain(q_raw, k_raw, v, gamma_q, gamma_k, grid, block, topk, rope_split=None, rope_theta=10000.0,
+                        eps=1e-6, softmax_scale=0.0, workspace=None, stream=None):
+    """The whole hot path on device tensors: prologue -> select -> attention.
+    Returns (o, lse, idx)."""
+    q, k = sol_qk_prologue(q_raw, k_raw, gamma_q, gamma_k, grid, rope_split, rope_theta, eps, stream=stream)
+    idx = sol_block_select(q, k, grid, block, topk, workspace=workspace, stream=stream)
+    o, lse = sol_sparse_attn_fwd(q, k, v, idx, grid, block, softmax_scale, stream=stream)
+    return o, lse, idx

@@ -1,0 +1,59 @@
+"""Builds libsol.so (the C-ABI library) in-tree with nvcc for sm_100a.
+
+    python -m block_sparse_attention_sol_b200.build [--verbose]
+
+One translation unit (csrc/sol_api.cu includes every kernel header), static
+CUDA runtime, no torch dependency: the library only needs the driver at run time.
+"""
+from __future__ import annotations
+
+import os
+import subprocess
+import sys
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(HERE)
+LIB = os.path.join(HERE, "libsol.so")
+SOURCES = [os.path.join(HERE, "csrc", "sol_api.cu")]
+NVCC_FLAGS = [
+    "-gencode", "arch=compute_100a,code=sm_100a",
+    "-O3", "-lineinfo", "-std=c++17",
+    "-Xcompiler", "-fPIC", "-shared",
+    "-Xptxas", "-warn-spills",
+]
+
+
+def nvcc() -> str:
+    for cand in (os.environ.get("NVCC"), "/usr/local/cuda/bin/nvcc"):
+        if cand and os.path.exists(cand):
+            return cand
+    return "nvcc"
+
+
+def _stale() -> bool:
+    if not os.path.exists(LIB):
+        return True
+    mtime = os.path.getmtime(LIB)
+    deps = [os.path.join(ROOT, "include", "sol.h"), __file__]
+    for d in os.listdir(os.path.join(HERE, "csrc")):
+        deps.append(os.path.join(HERE, "csrc", d))
+    return any(os.path.getmtime(p) > mtime for p in deps)
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    if not force and not _stale():
+        return LIB
+    cmd = [nvcc(), *NVCC_FLAGS, *(["-Xptxas", "-v"] if verbose else []), "-o", LIB + ".tmp", *SOURCES]
+    proc = subprocess.run(cmd, capture_output=True, text=True)
+    if proc.returncode != 0:
+        sys.stderr.write(proc.stdout + proc.stderr)
+        raise RuntimeError("nvcc failed building libsol.so")
+    if verbose:
+        sys.stderr.write(proc.stderr)
+    os.replace(LIB + ".tmp", LIB)
+    return LIB
+
+
+if __name__ == "__main__":
+    build(force=True, verbose="--verbose" in sys.argv)
+    print(LIB)

@@ -1,0 +1,304 @@
+// libsol: the C ABI declared in include/sol.h.
+//
+// Host side of every call: validate arguments (before any CUDA call, so that a
+// bad argument never launches anything), build TMA tensor maps where a kernel
+// needs them, size grids from the device's SM count, and launch on the
+// caller's stream.  Nothing here allocates device memory.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/sol.h"
+#include "sm100_ptx.cuh"
+#include "attn_f32.cuh"
+#include "attn_sm100.cuh"
+#include "prologue.cuh"
+#include "select.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool shape_ok(const sol_shape& s) {
+  if (s.B <= 0 || s.N <= 0 || s.H <= 0 || s.D <= 0) return false;
+  if (s.grid_t <= 0 || s.grid_h <= 0 || s.grid_w <= 0) return false;
+  const long long n = static_cast<long long>(s.grid_t) * s.grid_h * s.grid_w;
+  if (n != s.N) return false;
+  // every tensor is indexed with 64-bit offsets; keep each dimension product sane
+  const long long elems = static_cast<long long>(s.B) * s.N * s.H * s.D;
+  return elems > 0 && elems < (1ll << 40);
+}
+
+int num_blocks(int N, int block) { return (N + block - 1) / block; }
+
+struct DeviceInfo {
+  int sm_count = 0;
+  bool attn_attr = false, select_attr64 = false, select_attr128 = false;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+sol_status device_info(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SOL_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (d.sm_count == 0) {
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+      return SOL_ERR_CUDA;
+    d.sm_count = sms;
+  }
+  *out = &d;
+  return SOL_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<PFN_cuTensorMapEncodeTiled_v12000>(nullptr);
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }();
+  return fn;
+}
+
+// [B, N, H, D=128] bf16 viewed as a 4-D tensor (D, H, N, B); box = 64 channels x
+// 1 head x 128 tokens x 1 batch, 128-byte swizzle; tokens past N read as zero.
+sol_status make_bshd_map(CUtensorMap* map, const void* base, const sol_shape& s) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return SOL_ERR_CUDA;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(s.D), static_cast<cuuint64_t>(s.H), static_cast<cuuint64_t>(s.N),
+                        static_cast<cuuint64_t>(s.B)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(s.D) * 2, static_cast<cuuint64_t>(s.H) * s.D * 2,
+                           static_cast<cuuint64_t>(s.N) * s.H * s.D * 2};
+  cuuint32_t box[4] = {64, 1, 128, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? SOL_OK : SOL_ERR_CUDA;
+}
+
+sol_status launch_status() { return cudaGetLastError() == cudaSuccess ? SOL_OK : SOL_ERR_CUDA; }
+
+__global__ void wait_timeout_selftest_kernel(unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    sol::mbar_init(&bar, 1);
+    sol::fence_mbar_init();
+    // nothing ever arrives on `bar`: the bounded wait must give up and report
+    sol::mbar_wait(&bar, 0, &abort_flag, 0xFFu, limit_ns);
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* sol_status_string(sol_status st) {
+  switch (st) {
+    case SOL_OK: return "SOL_OK";
+    case SOL_ERR_INVALID_ARG: return "SOL_ERR_INVALID_ARG";
+    case SOL_ERR_UNSUPPORTED: return "SOL_ERR_UNSUPPORTED";
+    case SOL_ERR_CUDA: return "SOL_ERR_CUDA";
+    case SOL_ERR_TIMEOUT: return "SOL_ERR_TIMEOUT";
+  }
+  return "SOL_ERR_UNKNOWN";
+}
+
+sol_status sol_qk_prologue(const void* q_raw, const void* k_raw, void* q_out, void* k_out, const float* gamma_q,
+                           const float* gamma_k, sol_shape s, int rope_dt, int rope_dh, int rope_dw, float rope_theta,
+                           float eps, sol_dtype dt, cudaStream_t stream) {
+  if (!q_raw || !k_raw || !q_out || !k_out || !gamma_q || !gamma_k) return SOL_ERR_INVALID_ARG;
+  if (!aligned16(q_raw) || !aligned16(k_raw) || !aligned16(q_out) || !aligned16(k_out)) return SOL_ERR_INVALID_ARG;
+  if (!shape_ok(s)) return SOL_ERR_INVALID_ARG;
+  if (dt != SOL_F32 && dt != SOL_BF16) return SOL_ERR_INVALID_ARG;
+  if (rope_dt < 0 || rope_dh < 0 || rope_dw < 0 || (rope_dt | rope_dh | rope_dw) & 1) return SOL_ERR_INVALID_ARG;
+  if (rope_dt + rope_dh + rope_dw != s.D) return SOL_ERR_INVALID_ARG;
+  if (!(rope_theta > 0.f) || !(eps >= 0.f) || !std::isfinite(rope_theta) || !std::isfinite(eps))
+    return SOL_ERR_INVALID_ARG;
+  if (s.D != 64 && s.D != 128) return SOL_ERR_UNSUPPORTED;
+
+  sol::prologue::Params p;
+  p.q_in = q_raw; p.k_in = k_raw; p.q_out = q_out; p.k_out = k_out;
+  p.gamma_q = gamma_q; p.gamma_k = gamma_k;
+  p.rows = static_cast<long long>(s.B) * s.N * s.H;
+  p.N = s.N; p.H = s.H;
+  p.gt = s.grid_t; p.gh = s.grid_h; p.gw = s.grid_w;
+  p.dt = rope_dt; p.dh = rope_dh; p.dw = rope_dw;
+  p.log2_theta = std::log2(rope_theta);
+  p.eps = eps;
+  p.tab_t = s.grid_t * (rope_dt / 2);
+  p.tab_h = p.tab_t + s.grid_h * (rope_dh / 2);
+  p.tab_total = p.tab_h + s.grid_w * (rope_dw / 2);
+  const size_t smem = static_cast<size_t>(p.tab_total) * sizeof(float2);
+  if (smem > 48 * 1024) return SOL_ERR_UNSUPPORTED;
+
+  DeviceInfo* di = nullptr;
+  if (sol_status st = device_info(&di)) return st;
+  const int threads = 256;
+  const int lanes_per_row = (dt == SOL_BF16) ? s.D / 8 : s.D / 4;
+  const long long groups_needed = (p.rows + 0) * lanes_per_row / threads + 1;
+  const int grid = static_cast<int>(std::min<long long>(groups_needed, 8ll * di->sm_count));
+  if (dt == SOL_BF16) {
+    if (s.D == 128) sol::prologue::qk_prologue_kernel<__nv_bfloat16, 128><<<grid, threads, smem, stream>>>(p);
+    else sol::prologue::qk_prologue_kernel<__nv_bfloat16, 64><<<grid, threads, smem, stream>>>(p);
+  } else {
+    if (s.D == 128) sol::prologue::qk_prologue_kernel<float, 128><<<grid, threads, smem, stream>>>(p);
+    else sol::prologue::qk_prologue_kernel<float, 64><<<grid, threads, smem, stream>>>(p);
+  }
+  return launch_status();
+}
+
+size_t sol_block_select_workspace_bytes(sol_shape s, int block) {
+  if (!shape_ok(s) || block <= 0) return 0;
+  return 2ull * s.B * s.H * static_cast<size_t>(num_blocks(s.N, block)) * s.D * sizeof(float);
+}
+
+sol_status sol_block_select(const void* q, const void* k, sol_shape s, int block, int topk, sol_dtype dt,
+                            int32_t* idx_out, float* scores_out, void* workspace, size_t workspace_bytes,
+                            cudaStream_t stream) {
+  if (!q || !k || !idx_out || !workspace) return SOL_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(workspace) || !aligned16(idx_out)) return SOL_ERR_INVALID_ARG;
+  if (scores_out && !aligned16(scores_out)) return SOL_ERR_INVALID_ARG;
+  if (!shape_ok(s) || block <= 0) return SOL_ERR_INVALID_ARG;
+  if (dt != SOL_F32 && dt != SOL_BF16) return SOL_ERR_INVALID_ARG;
+  const int nb = num_blocks(s.N, block);
+  if (topk < 1 || topk > nb) return SOL_ERR_INVALID_ARG;
+  if (workspace_bytes < sol_block_select_workspace_bytes(s, block)) return SOL_ERR_INVALID_ARG;
+  if (s.D != 64 && s.D != 128) return SOL_ERR_UNSUPPORTED;
+  if (nb > 2048) return SOL_ERR_UNSUPPORTED;
+  if (static_cast<long long>(s.B) * s.H > 65535) return SOL_ERR_UNSUPPORTED;
+
+  DeviceInfo* di = nullptr;
+  if (sol_status st = device_info(&di)) return st;
+  float* qbar = static_cast<float*>(workspace);
+  float* kbar = qbar + static_cast<size_t>(s.B) * s.H * nb * s.D;
+  dim3 pg(nb, s.B, 2);
+  if (dt == SOL_BF16)
+    sol::select::block_pool_kernel<__nv_bfloat16><<<pg, 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), qbar, kbar, s.N, s.H, s.D, block,
+        nb);
+  else
+    sol::select::block_pool_kernel<float><<<pg, 256, 0, stream>>>(static_cast<const float*>(q),
+                                                                  static_cast<const float*>(k), qbar, kbar, s.N, s.H,
+                                                                  s.D, block, nb);
+  if (sol_status st = launch_status()) return st;
+
+  const size_t smem = (static_cast<size_t>(sol::select::kRows + sol::select::kKeys) * (s.D + 4) +
+                       static_cast<size_t>(sol::select::kRows) * nb) * sizeof(float);
+  dim3 sg((nb + sol::select::kRows - 1) / sol::select::kRows, s.B * s.H);
+  if (s.D == 128) {
+    if (!di->select_attr128) {
+      if (cudaFuncSetAttribute(sol::select::score_topk_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               200 * 1024) != cudaSuccess)
+        return SOL_ERR_CUDA;
+      di->select_attr128 = true;
+    }
+    sol::select::score_topk_kernel<128><<<sg, sol::select::kThreads, smem, stream>>>(qbar, kbar, idx_out, scores_out,
+                                                                                     nb, topk);
+  } else {
+    if (!di->select_attr64) {
+      if (cudaFuncSetAttribute(sol::select::score_topk_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               200 * 1024) != cudaSuccess)
+        return SOL_ERR_CUDA;
+      di->select_attr64 = true;
+    }
+    sol::select::score_topk_kernel<64><<<sg, sol::select::kThreads, smem, stream>>>(qbar, kbar, idx_out, scores_out,
+                                                                                    nb, topk);
+  }
+  return launch_status();
+}
+
+sol_status sol_sparse_attn_fwd(const void* q, const void* k, const void* v, const int32_t* idx, sol_shape s,
+                               int block, int topk, float softmax_scale, sol_dtype dt, void* o, float* lse,
+                               cudaStream_t stream) {
+  if (!q || !k || !v || !idx || !o || !lse) return SOL_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(idx) || !aligned16(lse))
+    return SOL_ERR_INVALID_ARG;
+  if (!shape_ok(s) || block <= 0) return SOL_ERR_INVALID_ARG;
+  if (dt != SOL_F32 && dt != SOL_BF16) return SOL_ERR_INVALID_ARG;
+  const int nb = num_blocks(s.N, block);
+  if (topk < 1 || topk > nb) return SOL_ERR_INVALID_ARG;
+  if (!std::isfinite(softmax_scale)) return SOL_ERR_INVALID_ARG;
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(s.D));
+
+  DeviceInfo* di = nullptr;
+  if (sol_status st = device_info(&di)) return st;
+
+  if (dt == SOL_F32) {
+    if (s.D != 64 && s.D != 128) return SOL_ERR_UNSUPPORTED;
+    const long long rows = static_cast<long long>(s.B) * s.H * s.N;
+    const long long grid = (rows + sol::attnf32::kWarps - 1) / sol::attnf32::kWarps;
+    if (grid > 0x7fffffffll) return SOL_ERR_UNSUPPORTED;
+    if (s.D == 128)
+      sol::attnf32::sparse_attn_fwd_f32_kernel<128><<<static_cast<int>(grid), sol::attnf32::kWarps * 32, 0, stream>>>(
+          static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v), idx,
+          static_cast<float*>(o), lse, s.B, s.N, s.H, block, nb, topk, scale);
+    else
+      sol::attnf32::sparse_attn_fwd_f32_kernel<64><<<static_cast<int>(grid), sol::attnf32::kWarps * 32, 0, stream>>>(
+          static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v), idx,
+          static_cast<float*>(o), lse, s.B, s.N, s.H, block, nb, topk, scale);
+    return launch_status();
+  }
+
+  // bf16: tcgen05 tensor-core path
+  if (s.D != sol::attn100::kHeadDim || block != sol::attn100::kBlock) return SOL_ERR_UNSUPPORTED;
+  const long long tiles = static_cast<long long>(s.B) * s.H * nb;
+  if (tiles > 0x7fffffffll) return SOL_ERR_UNSUPPORTED;
+  CUtensorMap tq, tk, tv;
+  if (sol_status st = make_bshd_map(&tq, q, s)) return st;
+  if (sol_status st = make_bshd_map(&tk, k, s)) return st;
+  if (sol_status st = make_bshd_map(&tv, v, s)) return st;
+  const size_t smem = sizeof(sol::attn100::Smem) + 1024;
+  if (!di->attn_attr) {
+    if (cudaFuncSetAttribute(sol::attn100::sparse_attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return SOL_ERR_CUDA;
+    di->attn_attr = true;
+  }
+  sol::attn100::Params p;
+  p.idx = idx;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.B = s.B; p.N = s.N; p.H = s.H; p.nb = nb; p.topk = topk;
+  p.num_tiles = static_cast<int>(tiles);
+  p.scale_log2 = scale * 1.4426950408889634f;
+  const int grid = static_cast<int>(std::min<long long>(tiles, di->sm_count));
+  sol::attn100::sparse_attn_fwd_kernel<<<grid, sol::attn100::kThreads, smem, stream>>>(tq, tk, tv, p);
+  return launch_status();
+}
+
+sol_status sol_check_device_status(cudaStream_t stream) {
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return SOL_ERR_CUDA;
+  unsigned int word = 0;
+  if (cudaMemcpyFromSymbol(&word, sol::g_error_word, sizeof(word)) != cudaSuccess) return SOL_ERR_CUDA;
+  if (word != 0u) {
+    const unsigned int zero = 0u;
+    if (cudaMemcpyToSymbol(sol::g_error_word, &zero, sizeof(zero)) != cudaSuccess) return SOL_ERR_CUDA;
+    return (word & sol::kErrTimeout) ? SOL_ERR_TIMEOUT : SOL_ERR_INVALID_ARG;
+  }
+  return SOL_OK;
+}
+
+sol_status sol_selftest_wait_timeout(unsigned limit_us, cudaStream_t stream) {
+  if (limit_us < 1u || limit_us > 1000000u) return SOL_ERR_INVALID_ARG;
+  wait_timeout_selftest_kernel<<<1, 32, 0, stream>>>(static_cast<unsigned long long>(limit_us) * 1000ull);
+  return launch_status();
+}
+
+}  // extern "C"

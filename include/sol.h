@@ -1,0 +1,141 @@
+/*
+ * sol.h -- C ABI of libsol, the B200 (sm_100a) implementation of the Sol-Attn
+ * hot path: fused QK-RMSNorm + 3D RoPE, block selection, and block-sparse
+ * attention returning O and LSE.
+ *
+ * Source of the method.  The Sol-H3 runtime for MiniMax-H3 video diffusion
+ * credits Sol-Attn -- a training-free sparse attention that decides per query
+ * which parts of the attention computation matter -- with the largest share of
+ * its speed-up, and merges normalisation and RoPE into single kernels
+ * (ai-feiten.nl, "Videomodel MiniMax-H3 rendert sneller dan afspelen", section
+ * "Waar de snelheidswinst vandaan komt").  The pages give no formulas; the
+ * concrete definition implemented here is stated at each call.
+ *
+ * Conventions shared by every call
+ *  - Layouts: activations are [B, N, H, D] contiguous ("BSHD": token-major,
+ *    then head, then channel).  Tokens are the latent video grid
+ *    (grid_t, grid_h, grid_w) flattened in raster order, n = (t*grid_h + y)*grid_w + x.
+ *    Blocks are runs of `block` consecutive tokens; the last may be short.
+ *  - Memory: every pointer is a DEVICE pointer on the current CUDA device,
+ *    16-byte aligned, owned by the caller.  The library never allocates,
+ *    frees or synchronises, except sol_check_device_status(), which
+ *    synchronises its stream.
+ *  - Asynchrony: work is enqueued on `stream` and returns immediately.
+ *    Argument errors are reported synchronously (SOL_ERR_INVALID_ARG /
+ *    SOL_ERR_UNSUPPORTED) before anything is launched; launch failures return
+ *    SOL_ERR_CUDA.  Device-side waits are bounded (2 s); a wait that runs out
+ *    sets a device error word that sol_check_device_status() reports as
+ *    SOL_ERR_TIMEOUT.
+ *  - Thread safety: stateless apart from that error word and per-device
+ *    caches of kernel attributes; calls may come from several host threads.
+ */
+#ifndef SOL_H_
+#define SOL_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SOL_OK = 0,
+  SOL_ERR_INVALID_ARG = 1,   /* null / misaligned pointer, inconsistent shape, k out of range */
+  SOL_ERR_UNSUPPORTED = 2,   /* valid request outside the implemented shapes / dtypes          */
+  SOL_ERR_CUDA = 3,          /* a CUDA runtime or driver call failed                            */
+  SOL_ERR_TIMEOUT = 4        /* a device-side bounded wait ran out (see sol_check_device_status) */
+} sol_status;
+
+typedef enum { SOL_F32 = 0, SOL_BF16 = 1 } sol_dtype;
+
+/* B batch, N tokens (== grid_t*grid_h*grid_w), H heads, D head dim. */
+typedef struct {
+  int B, N, H, D;
+  int grid_t, grid_h, grid_w;
+} sol_shape;
+
+/*
+ * sol_qk_prologue -- fused QK-RMSNorm + 3D RoPE (normalisation and RoPE merged
+ * into one kernel: ai-feiten.nl, "Videomodel MiniMax-H3 rendert sneller dan
+ * afspelen", "Waar de snelheidswinst vandaan komt").
+ *
+ * For Q and K, per (b, n, h):
+ *   y_d = x_d / sqrt(mean_d x_d^2 + eps) * gamma[h*D + d]
+ *   then channel pairs (2p, 2p+1) rotate by angle pos * theta^(-2i/d_axis):
+ *   the first rope_dt/2 pairs use the frame index t, the next rope_dh/2 the row
+ *   y, the last rope_dw/2 the column x; i counts pairs within the axis.
+ *   (y0, y1) -> (y0 cos - y1 sin, y0 sin + y1 cos).
+ * q_raw, k_raw : [B,N,H,D] inputs (dtype dt);  q_out, k_out : [B,N,H,D] outputs
+ *                (may alias the inputs exactly, not partially).
+ * gamma_q, gamma_k : fp32 [H*D].
+ * rope_dt + rope_dh + rope_dw == D, each even.  D in {64, 128}.
+ * Arithmetic in fp32; bf16 outputs are rounded to nearest even.
+ */
+sol_status sol_qk_prologue(const void* q_raw, const void* k_raw, void* q_out, void* k_out,
+                           const float* gamma_q, const float* gamma_k, sol_shape s,
+                           int rope_dt, int rope_dh, int rope_dw, float rope_theta, float eps,
+                           sol_dtype dt, cudaStream_t stream);
+
+/* Bytes of scratch sol_block_select needs: the fp32 pooled means of Q and K,
+ * 2 * B * H * ceil(N/block) * D * 4.  Returns 0 for an invalid shape. */
+size_t sol_block_select_workspace_bytes(sol_shape s, int block);
+
+/*
+ * sol_block_select -- the "preparation" of the sparse attention
+ * (ai-feiten.nl, same section: it became 76.4% faster in Sol-H3).
+ *
+ * qbar[b,h,i] = mean of q over the valid tokens of block i (likewise kbar);
+ * s[b,h,i,j]  = qbar[b,h,i] . kbar[b,h,j]  (fp32);
+ * idx[b,h,i,:] = the topk largest s[b,h,i,:], exact ties to the lower j,
+ *                listed in ascending j.
+ * q, k        : [B,N,H,D] (dtype dt), normally sol_qk_prologue's outputs.
+ * idx_out     : int32 [B, H, nb, topk], nb = ceil(N/block).
+ * scores_out  : optional fp32 [B, H, nb, nb] copy of s (NULL to skip).
+ * workspace   : device scratch of at least sol_block_select_workspace_bytes().
+ * 1 <= topk <= nb, D in {64, 128}, nb <= 2048.
+ */
+sol_status sol_block_select(const void* q, const void* k, sol_shape s, int block, int topk,
+                            sol_dtype dt, int32_t* idx_out, float* scores_out,
+                            void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * sol_sparse_attn_fwd -- Sol-Attn block-sparse attention forward
+ * (ai-feiten.nl, same section: attention restricted, per query, to the parts
+ * that matter).
+ *
+ * For each query n of block i of (b, h), over the keys m < N of the blocks
+ * idx[b,h,i,0..topk-1]:
+ *   l_m = scale * q_n . k_m;  o_n = sum_m softmax(l)_m v_m;  lse_n = ln sum_m exp(l_m).
+ * q, k, v : [B,N,H,D] (dtype dt).  idx : int32 [B,H,nb,topk], distinct ids in
+ *           [0, nb) per row (any order; not checked).
+ * o       : [B,N,H,D] (dtype dt).  lse : fp32 [B,H,N], natural log, scale included.
+ * softmax_scale <= 0 selects 1/sqrt(D).
+ * bf16: D == 128 and block == 128 (tcgen05 tensor-core kernel, fp32 accumulate,
+ *       P rounded to bf16 for the PV product).
+ * f32 : D in {64, 128}, any block (CUDA-core kernel, fp32 throughout).
+ */
+sol_status sol_sparse_attn_fwd(const void* q, const void* k, const void* v, const int32_t* idx,
+                               sol_shape s, int block, int topk, float softmax_scale,
+                               sol_dtype dt, void* o, float* lse, cudaStream_t stream);
+
+/* Synchronises `stream`, then reads and clears the device error word.
+ * Returns SOL_ERR_TIMEOUT if a bounded device wait ran out since the last
+ * check, SOL_ERR_CUDA if the stream reports a CUDA error, else SOL_OK. */
+sol_status sol_check_device_status(cudaStream_t stream);
+
+/* Launches one thread that waits on a barrier nothing will complete, bounded
+ * by limit_us (1..1000000) microseconds, so that the timeout path can be
+ * exercised without a hang.  The following sol_check_device_status() on the
+ * same stream returns SOL_ERR_TIMEOUT.  No counterpart on the pages: this is a
+ * self-test of the library's failure detection. */
+sol_status sol_selftest_wait_timeout(unsigned limit_us, cudaStream_t stream);
+
+/* Static, human-readable name of a status code. */
+const char* sol_status_string(sol_status status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SOL_H_ */

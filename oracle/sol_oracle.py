@@ -82,21 +82,25 @@ def rope_angles(grid, split, theta: float) -> np.ndarray:
     return np.stack(cols, axis=1)
 
 
-def qk_prologue(x, gamma, grid, split, theta: float, eps: float) -> np.ndarray:
+def qk_prologue(x, gamma, grid, split, theta: float, eps: float, tokens=None) -> np.ndarray:
     """Fused QK-RMSNorm + 3D RoPE of one tensor (Q or K), float64 result.
 
     x: [B, N, H, D] (any float dtype, widened exactly); gamma: [H*D].
+    tokens: optional token indices; then only those rows are computed and the
+    result is [B, len(tokens), H, D].
     y = x / sqrt(mean_d x^2 + eps) * gamma[h, d]; then each pair (y0, y1) of a
     token turns by its angle phi: (y0 cos phi - y1 sin phi, y0 sin phi + y1 cos phi).
     Reading: the norm runs over the head dimension of one (token, head); RMSNorm
     comes before RoPE; V is not touched.  The caller rounds to the stored dtype.
     """
-    x = np.asarray(x, dtype=np.float64)
     B, N, H, D = x.shape
+    x = np.asarray(x if tokens is None else x[:, tokens], dtype=np.float64)
     g = np.asarray(gamma, dtype=np.float64).reshape(H, D)
     rms = np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)
     y = x / rms * g[None, None, :, :]
     phi = rope_angles(grid, split, theta)                   # [N, D/2]
+    if tokens is not None:
+        phi = phi[tokens]
     c = np.cos(phi)[None, :, None, :]
     s = np.sin(phi)[None, :, None, :]
     y0 = y[..., 0::2]
@@ -113,12 +117,11 @@ def block_pool(x, block: int) -> np.ndarray:
     Reading: blocks are runs of consecutive raster-order tokens; the last block
     may be short (N % block tokens) and is averaged over its valid tokens only.
     """
-    x = np.asarray(x, dtype=np.float64)
     B, N, H, D = x.shape
     nb = -(-N // block)
     out = np.empty((B, H, nb, D))
     for i in range(nb):
-        seg = x[:, i * block:min(N, (i + 1) * block)]       # [B, n_i, H, D]
+        seg = np.asarray(x[:, i * block:min(N, (i + 1) * block)], dtype=np.float64)   # [B, n_i, H, D]
         out[:, :, i, :] = seg.mean(axis=1)
     return out
 

@@ -1,0 +1,113 @@
+"""Host-side checks of the C-ABI library that need no GPU: it loads, exports
+every symbol include/sol.h declares, and rejects bad arguments synchronously
+(before any CUDA call is made)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sol.h")
+LIB = os.path.join(ROOT, "block_sparse_attention_sol_b200", "libsol.so")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(LIB):
+        from block_sparse_attention_sol_b200.build import build
+        build()
+    return ctypes.CDLL(LIB)
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sol_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_three_calls():
+    names = declared_functions()
+    for n in ("sol_qk_prologue", "sol_block_select", "sol_sparse_attn_fwd", "sol_check_device_status"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in ("B", "N", "H", "D", "grid_t", "grid_h", "grid_w")]
+
+
+FAKE = ctypes.c_void_p(0x10000)      # aligned, never dereferenced on the host
+MISALIGNED = ctypes.c_void_p(0x10008)
+OK_SHAPE = Shape(1, 1024, 2, 64, 4, 16, 16)
+INVALID, UNSUPPORTED = 1, 2
+
+
+def prologue(lib, shape=OK_SHAPE, split=(24, 20, 20), ptr=FAKE, theta=10000.0, eps=1e-6, dt=0):
+    f = lib.sol_qk_prologue
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p] * 6 + [Shape, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float,
+                                          ctypes.c_float, ctypes.c_int, ctypes.c_void_p]
+    return f(ptr, FAKE, FAKE, FAKE, FAKE, FAKE, shape, *split, theta, eps, dt, None)
+
+
+def test_prologue_argument_checks(lib):
+    assert prologue(lib, ptr=None) == INVALID
+    assert prologue(lib, ptr=MISALIGNED) == INVALID
+    assert prologue(lib, split=(24, 20, 18)) == INVALID          # does not sum to D
+    assert prologue(lib, split=(23, 21, 20)) == INVALID          # odd
+    assert prologue(lib, shape=Shape(1, 1000, 2, 64, 4, 16, 16)) == INVALID   # N != grid product
+    assert prologue(lib, theta=0.0) == INVALID
+    assert prologue(lib, eps=-1.0) == INVALID
+    assert prologue(lib, dt=7) == INVALID
+    assert prologue(lib, shape=Shape(1, 1024, 2, 96, 4, 16, 16), split=(32, 32, 32)) == UNSUPPORTED
+
+
+def test_select_argument_checks(lib):
+    f = lib.sol_block_select
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p, ctypes.c_void_p, Shape, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                  ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+    wsb = lib.sol_block_select_workspace_bytes
+    wsb.restype = ctypes.c_size_t
+    wsb.argtypes = [Shape, ctypes.c_int]
+    need = wsb(OK_SHAPE, 64)
+    assert need == 2 * 1 * 2 * 16 * 64 * 4
+    assert wsb(Shape(1, 1000, 2, 64, 4, 16, 16), 64) == 0
+    assert f(FAKE, FAKE, OK_SHAPE, 64, 0, 0, FAKE, None, FAKE, need, None) == INVALID        # k = 0
+    assert f(FAKE, FAKE, OK_SHAPE, 64, 17, 0, FAKE, None, FAKE, need, None) == INVALID       # k > nb
+    assert f(FAKE, FAKE, OK_SHAPE, 64, 4, 0, FAKE, None, FAKE, need - 4, None) == INVALID    # small workspace
+    assert f(FAKE, FAKE, OK_SHAPE, 64, 4, 0, None, None, FAKE, need, None) == INVALID        # no idx_out
+    assert f(FAKE, FAKE, OK_SHAPE, 0, 4, 0, FAKE, None, FAKE, need, None) == INVALID         # block 0
+
+
+def test_attention_argument_checks(lib):
+    f = lib.sol_sparse_attn_fwd
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p] * 4 + [Shape, ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_int,
+                                          ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+    assert f(FAKE, FAKE, FAKE, FAKE, OK_SHAPE, 64, 0, 0.0, 0, FAKE, FAKE, None) == INVALID
+    assert f(FAKE, FAKE, FAKE, FAKE, OK_SHAPE, 64, 17, 0.0, 0, FAKE, FAKE, None) == INVALID
+    assert f(FAKE, FAKE, None, FAKE, OK_SHAPE, 64, 4, 0.0, 0, FAKE, FAKE, None) == INVALID
+    assert f(FAKE, FAKE, FAKE, MISALIGNED, OK_SHAPE, 64, 4, 0.0, 0, FAKE, FAKE, None) == INVALID
+    assert f(FAKE, FAKE, FAKE, FAKE, OK_SHAPE, 64, 4, float("nan"), 0, FAKE, FAKE, None) == INVALID
+
+
+def test_selftest_limit_checked(lib):
+    f = lib.sol_selftest_wait_timeout
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_uint, ctypes.c_void_p]
+    assert f(0, None) == INVALID
+    assert f(2_000_000, None) == INVALID
+
+
+def test_status_strings(lib):
+    f = lib.sol_status_string
+    f.restype = ctypes.c_char_p
+    f.argtypes = [ctypes.c_int]
+    assert [f(i).decode() for i in range(5)] == ["SOL_OK", "SOL_ERR_INVALID_ARG", "SOL_ERR_UNSUPPORTED",
+                                                 "SOL_ERR_CUDA", "SOL_ERR_TIMEOUT"]
