@@ -6,7 +6,7 @@ import pytest
 import torch
 
 import oracle as orc
-from tests.gpu_common import (bf16_ulps, check_attention, check_selection, np32, np64, REL_TOL_F32)
+from tests.gpu_common import (check_bf16_prologue, check_attention, check_selection, np32, np64, REL_TOL_F32)
 from workloads import random_index_lists, rope_split_for
 
 pytestmark = pytest.mark.gpu
@@ -33,7 +33,7 @@ def test_prologue_small(sol, dtype, D, grid, H, B):
     for raw, g, out in ((q_raw, gq, q), (k_raw, gk, k)):
         ref = orc.qk_prologue(np64(raw), g.double().numpy(), grid, split, 10000.0, 1e-6)
         if dtype == torch.bfloat16:
-            assert bf16_ulps(np32(out), ref).max() <= 1
+            check_bf16_prologue(np32(out), ref)
         else:
             assert np.abs(np64(out) - ref).max() <= REL_TOL_F32 * np.abs(ref).max()
 
