@@ -45,16 +45,30 @@ def load_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+KERNEL_SOURCES = ("block_sparse_attention_sol_b200/csrc/attn_sm100.cuh",
+                  "block_sparse_attention_sol_b200/csrc/sm100_ptx.cuh")
+
+
 def load_ncu_traffic(kernel: str):
-    """Per-launch DRAM bytes of `kernel` from the committed ncu summary, or None."""
+    """Per-launch DRAM bytes of `kernel` from the committed ncu summary, or None
+    when there is none or the kernel sources changed since it was measured."""
+    import hashlib
     path = os.path.join(ROOT, "profiles", f"{kernel}_traffic.txt")
     if not os.path.exists(path):
         return None
+    h = hashlib.sha256()
+    for src in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, src), "rb") as f:
+            h.update(f.read())
+    fields = {}
     with open(path) as f:
         for line in f:
-            if line.startswith("dram_bytes_per_launch:"):
-                return float(line.split(":", 1)[1].split()[0])
-    return None
+            if ":" in line and not line.startswith("#"):
+                key, val = line.split(":", 1)
+                fields[key.strip()] = val.strip()
+    if fields.get("kernel_source_sha256") != h.hexdigest():
+        return None
+    return float(fields["dram_bytes_per_launch"])
 
 
 class ClockSampler:
@@ -260,7 +274,7 @@ def run_ours(args, wl, world, rank, local):
 
     # end to end through host buffers
     e2e_start, e2e_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e2e_steps = args.e2e_steps or args.steps
+    e2e_steps = 1 if args.no_e2e else (args.e2e_steps or args.steps)
     barrier(world)
     torch.cuda.synchronize(dev)
     e2e_start.record(stream)
@@ -314,8 +328,8 @@ def run_ours(args, wl, world, rank, local):
                           "frac_bf16": achieved / peaks["bf16_tflops"]},
             "hbm_peak_gbs": peaks["hbm_gbs"],
         },
-        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": e2e_ms},
+        "e2e": None if args.no_e2e else {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                                         "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": 4 * args.steps,
         "clocks": clocks,
     }
@@ -339,6 +353,7 @@ def main():
     ap.add_argument("--cpu-units", type=int, default=48)
     ap.add_argument("--ref-units", type=int, default=24)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="profiling runs: one e2e step, not reported")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -30,7 +30,7 @@ __all__ = [
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsol.so")
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m block_sparse_attention_sol_b200.build` "
+        f"{LIB_PATH} is missing: build it with `python block_sparse_attention_sol_b200/build.py` "
         "(there is no non-CUDA fallback)")
 lib = ctypes.CDLL(LIB_PATH)
 

@@ -1,6 +1,6 @@
 """Builds libsol.so (the C-ABI library) in-tree with nvcc for sm_100a.
 
-    python -m block_sparse_attention_sol_b200.build [--verbose]
+    python block_sparse_attention_sol_b200/build.py [--verbose]
 
 One translation unit (csrc/sol_api.cu includes every kernel header), static
 CUDA runtime, no torch dependency: the library only needs the driver at run time.
@@ -8,6 +8,7 @@ CUDA runtime, no torch dependency: the library only needs the driver at run time
 from __future__ import annotations
 
 import os
+import re
 import subprocess
 import sys
 
@@ -40,16 +41,36 @@ def _stale() -> bool:
     return any(os.path.getmtime(p) > mtime for p in deps)
 
 
+# Kernels whose spilling would silently cost performance: the build refuses them.
+NO_SPILL_KERNELS = ("sparse_attn_fwd_kernel",)
+
+
+def _check_ptxas_report(report: str) -> None:
+    lines = report.splitlines()
+    for name in NO_SPILL_KERNELS:
+        found = False
+        for i, line in enumerate(lines):
+            if "Compiling entry function" in line and name in line:
+                found = True
+                for follow in lines[i + 1:i + 4]:
+                    m = re.search(r"(\d+) bytes spill stores", follow)
+                    if m and int(m.group(1)) != 0:
+                        raise RuntimeError(f"{name} spills registers: {follow.strip()}")
+        if not found:
+            raise RuntimeError(f"no ptxas report for {name}")
+
+
 def build(force: bool = False, verbose: bool = False) -> str:
     if not force and not _stale():
         return LIB
-    cmd = [nvcc(), *NVCC_FLAGS, *(["-Xptxas", "-v"] if verbose else []), "-o", LIB + ".tmp", *SOURCES]
+    cmd = [nvcc(), *NVCC_FLAGS, "-Xptxas", "-v", "-o", LIB + ".tmp", *SOURCES]
     proc = subprocess.run(cmd, capture_output=True, text=True)
     if proc.returncode != 0:
         sys.stderr.write(proc.stdout + proc.stderr)
         raise RuntimeError("nvcc failed building libsol.so")
     if verbose:
         sys.stderr.write(proc.stderr)
+    _check_ptxas_report(proc.stderr)
     os.replace(LIB + ".tmp", LIB)
     return LIB
 

@@ -9,11 +9,14 @@
 // with the first dt/2 pairs on the frame axis t, the next dh/2 on the row axis
 // y and the last dw/2 on the column axis x; i is the pair index within its axis.
 //
-// HBM-bound streaming kernel: each group of D/VEC lanes owns one row and moves
-// it with 16-byte vector loads and stores; the sum of squares is reduced with
-// warp shuffles inside the group.  The per-axis cos/sin tables (a few KB) are
-// built once per CTA in shared memory, so the trigonometry is amortised over all
-// heads and tokens the CTA streams.  Arithmetic in fp32.
+// HBM-bound streaming kernel.  A group of D/VEC lanes owns one row and moves it
+// with 16-byte loads and stores; the sum of squares is reduced with shuffles
+// inside the group.  The grid holds a multiple of H groups, so every group keeps
+// one head for its whole life: its gains and its channel -> (axis, pair) map sit
+// in registers, and the loop advances by whole tokens with 32-bit indices.  Two
+// tokens are in flight per iteration.  The per-axis cos/sin tables (a few KB)
+// are built once per CTA in shared memory from double-precision angles, so the
+// rotation carries no angle error beyond rounding the table to fp32.
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -28,11 +31,11 @@ struct Params {
   void* k_out;
   const float* gamma_q;
   const float* gamma_k;
-  long long rows;        // B * N * H
+  int tokens;            // B * N
   int N, H;
   int gt, gh, gw;        // latent grid (T, Hg, Wg)
   int dt, dh, dw;        // rotary channels per axis
-  float log2_theta;
+  double log2_theta;
   float eps;
   int tab_t, tab_h;      // offsets (in float2) of the y and x tables in shared memory
   int tab_total;
@@ -48,65 +51,45 @@ __device__ __forceinline__ void load_vec(const float* p, float (&x)[4]) {
 }
 __device__ __forceinline__ void load_vec(const __nv_bfloat16* p, float (&x)[8]) {
   const uint4 v = __ldcs(reinterpret_cast<const uint4*>(p));
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    x[2 * i] = __uint_as_float(w[i] << 16);
-    x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-  }
+  x[0] = __uint_as_float(v.x << 16); x[1] = __uint_as_float(v.x & 0xFFFF0000u);
+  x[2] = __uint_as_float(v.y << 16); x[3] = __uint_as_float(v.y & 0xFFFF0000u);
+  x[4] = __uint_as_float(v.z << 16); x[5] = __uint_as_float(v.z & 0xFFFF0000u);
+  x[6] = __uint_as_float(v.w << 16); x[7] = __uint_as_float(v.w & 0xFFFF0000u);
 }
 __device__ __forceinline__ void store_vec(float* p, const float (&y)[4]) {
   *reinterpret_cast<float4*>(p) = make_float4(y[0], y[1], y[2], y[3]);
 }
+__device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
 __device__ __forceinline__ void store_vec(__nv_bfloat16* p, const float (&y)[8]) {
-  uint32_t w[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const __nv_bfloat162 b = __floats2bfloat162_rn(y[2 * i], y[2 * i + 1]);   // .x = low half
-    w[i] = *reinterpret_cast<const uint32_t*>(&b);
-  }
-  *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+  *reinterpret_cast<uint4*>(p) =
+      make_uint4(bf16x2_bits(y[0], y[1]), bf16x2_bits(y[2], y[3]), bf16x2_bits(y[4], y[5]), bf16x2_bits(y[6], y[7]));
 }
 
-// One row: normalise, scale by gamma, rotate.  `lane_in_row` owns channels
-// [lane_in_row*V, lane_in_row*V + V).
-template <typename T, int D>
-__device__ __forceinline__ void process_row(const T* in, T* out, const float* gamma, int h, const float2* tab_t,
-                                            const float2* tab_y, const float2* tab_x, int dt, int dh, float eps,
-                                            int lane_in_row) {
-  constexpr int V = Vec<T>::n;
-  constexpr int L = D / V;   // lanes per row
-  float x[V];
-  load_vec(in + lane_in_row * V, x);
+// Normalise, scale by the gains, rotate the V/2 channel pairs this lane owns.
+template <int V, int L>
+__device__ __forceinline__ void norm_rotate(float (&x)[V], const float (&g)[V], const float2 (&cs)[V / 2],
+                                            unsigned seg, int D, float eps) {
   float ss = 0.f;
 #pragma unroll
   for (int e = 0; e < V; ++e) ss = fmaf(x[e], x[e], ss);
-  // only the L lanes of this row's group take part (rows may run out unevenly in a warp)
-  const unsigned lane = threadIdx.x & 31u;
-  const unsigned seg = (L == 32) ? 0xffffffffu : (((1u << (L & 31)) - 1u) << (lane & ~(unsigned)(L - 1)));
 #pragma unroll
   for (int off = L / 2; off > 0; off >>= 1) ss += __shfl_xor_sync(seg, ss, off, L);
   const float r = 1.0f / sqrtf(ss / static_cast<float>(D) + eps);
-  const float* g = gamma + h * D + lane_in_row * V;
-  float y[V];
 #pragma unroll
   for (int e = 0; e < V; e += 2) {
-    const float y0 = x[e] * r * __ldg(g + e);
-    const float y1 = x[e + 1] * r * __ldg(g + e + 1);
-    const int c = lane_in_row * V + e;   // even channel index
-    float2 cs;
-    if (c < dt) cs = tab_t[c >> 1];
-    else if (c < dt + dh) cs = tab_y[(c - dt) >> 1];
-    else cs = tab_x[(c - dt - dh) >> 1];
-    y[e] = y0 * cs.x - y1 * cs.y;
-    y[e + 1] = y0 * cs.y + y1 * cs.x;
+    const float y0 = x[e] * r * g[e];
+    const float y1 = x[e + 1] * r * g[e + 1];
+    x[e] = y0 * cs[e / 2].x - y1 * cs[e / 2].y;
+    x[e + 1] = y0 * cs[e / 2].y + y1 * cs[e / 2].x;
   }
-  store_vec(out + lane_in_row * V, y);
 }
 
-// Grid-stride over rows; both Q and K rows are handled in the same iteration.
 template <typename T, int D>
-__global__ void __launch_bounds__(256) qk_prologue_kernel(const Params p) {
+__global__ void __launch_bounds__(256, sizeof(T) == 2 ? 3 : 4) qk_prologue_kernel(const Params p) {
   extern __shared__ float2 tab[];   // [gt * dt/2 | gh * dh/2 | gw * dw/2] of (cos, sin)
   const int pt = p.dt / 2, ph = p.dh / 2, pw = p.dw / 2;
   for (int i = threadIdx.x; i < p.tab_total; i += blockDim.x) {
@@ -114,33 +97,87 @@ __global__ void __launch_bounds__(256) qk_prologue_kernel(const Params p) {
     if (i < p.tab_t) { pos = i / pt; pair = i % pt; d_axis = p.dt; }
     else if (i < p.tab_h) { pos = (i - p.tab_t) / ph; pair = (i - p.tab_t) % ph; d_axis = p.dh; }
     else { pos = (i - p.tab_h) / pw; pair = (i - p.tab_h) % pw; d_axis = p.dw; }
-    const float inv_freq = exp2f(-p.log2_theta * (2.0f * pair) / static_cast<float>(d_axis));
-    float s, c;
-    sincosf(static_cast<float>(pos) * inv_freq, &s, &c);
-    tab[i] = make_float2(c, s);
+    const double angle = static_cast<double>(pos) * exp2(-p.log2_theta * (2.0 * pair) / d_axis);
+    double s, c;
+    sincos(angle, &s, &c);
+    tab[i] = make_float2(static_cast<float>(c), static_cast<float>(s));
   }
   __syncthreads();
 
   constexpr int V = Vec<T>::n;
-  constexpr int L = D / V;
+  constexpr int L = D / V;            // lanes per row
+  constexpr int GPC = 256 / L;        // row groups per CTA
   const int lane_in_row = threadIdx.x % L;
-  const long long group = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) / L;
-  const long long groups = static_cast<long long>(gridDim.x) * blockDim.x / L;
+  const unsigned lane = threadIdx.x & 31u;
+  const unsigned seg = (L == 32) ? 0xffffffffu : (((1u << (L & 31)) - 1u) << (lane & ~(unsigned)(L - 1)));
+  const int grp = blockIdx.x * GPC + threadIdx.x / L;
+  const int groups = gridDim.x * GPC;          // a multiple of H (host guarantees)
+  const int h = grp % p.H;
+  const int tok_step = groups / p.H;
+
+  // per-lane constants: gains and the table slot (axis, pair) of each owned channel pair
+  float gq[V], gk[V];
+#pragma unroll
+  for (int e = 0; e < V; ++e) {
+    gq[e] = __ldg(p.gamma_q + h * D + lane_in_row * V + e);
+    gk[e] = __ldg(p.gamma_k + h * D + lane_in_row * V + e);
+  }
+  int axis[V / 2], slot[V / 2];
+#pragma unroll
+  for (int e = 0; e < V / 2; ++e) {
+    const int c = lane_in_row * V + 2 * e;
+    if (c < p.dt) { axis[e] = 0; slot[e] = c / 2; }
+    else if (c < p.dt + p.dh) { axis[e] = 1; slot[e] = p.tab_t + (c - p.dt) / 2; }
+    else { axis[e] = 2; slot[e] = p.tab_h + (c - p.dt - p.dh) / 2; }
+  }
+
   const T* qi = static_cast<const T*>(p.q_in);
   const T* ki = static_cast<const T*>(p.k_in);
   T* qo = static_cast<T*>(p.q_out);
   T* ko = static_cast<T*>(p.k_out);
   const int hw = p.gh * p.gw;
-  for (long long row = group; row < p.rows; row += groups) {
-    const int h = static_cast<int>(row % p.H);
-    const int n = static_cast<int>((row / p.H) % p.N);
+
+  auto angles = [&](int tok, float2 (&cs)[V / 2]) {
+    const int n = tok % p.N;
     const int t = n / hw, y = (n / p.gw) % p.gh, x = n % p.gw;
-    const float2* tt = tab + t * pt;
-    const float2* ty = tab + p.tab_t + y * ph;
-    const float2* tx = tab + p.tab_h + x * pw;
-    const size_t off = static_cast<size_t>(row) * D;
-    process_row<T, D>(qi + off, qo + off, p.gamma_q, h, tt, ty, tx, p.dt, p.dh, p.eps, lane_in_row);
-    process_row<T, D>(ki + off, ko + off, p.gamma_k, h, tt, ty, tx, p.dt, p.dh, p.eps, lane_in_row);
+    const int st = t * pt, sy = y * ph, sx = x * pw;
+#pragma unroll
+    for (int e = 0; e < V / 2; ++e) cs[e] = tab[slot[e] + (axis[e] == 0 ? st : (axis[e] == 1 ? sy : sx))];
+  };
+
+  int tok = grp / p.H;
+  for (; tok + tok_step < p.tokens; tok += 2 * tok_step) {
+    const int tok2 = tok + tok_step;
+    const size_t o1 = (static_cast<size_t>(tok) * p.H + h) * D + lane_in_row * V;
+    const size_t o2 = (static_cast<size_t>(tok2) * p.H + h) * D + lane_in_row * V;
+    float xq1[V], xk1[V], xq2[V], xk2[V];
+    load_vec(qi + o1, xq1);
+    load_vec(ki + o1, xk1);
+    load_vec(qi + o2, xq2);
+    load_vec(ki + o2, xk2);
+    float2 cs1[V / 2], cs2[V / 2];
+    angles(tok, cs1);
+    angles(tok2, cs2);
+    norm_rotate<V, L>(xq1, gq, cs1, seg, D, p.eps);
+    norm_rotate<V, L>(xk1, gk, cs1, seg, D, p.eps);
+    norm_rotate<V, L>(xq2, gq, cs2, seg, D, p.eps);
+    norm_rotate<V, L>(xk2, gk, cs2, seg, D, p.eps);
+    store_vec(qo + o1, xq1);
+    store_vec(ko + o1, xk1);
+    store_vec(qo + o2, xq2);
+    store_vec(ko + o2, xk2);
+  }
+  if (tok < p.tokens) {
+    const size_t o1 = (static_cast<size_t>(tok) * p.H + h) * D + lane_in_row * V;
+    float xq[V], xk[V];
+    load_vec(qi + o1, xq);
+    load_vec(ki + o1, xk);
+    float2 cs[V / 2];
+    angles(tok, cs);
+    norm_rotate<V, L>(xq, gq, cs, seg, D, p.eps);
+    norm_rotate<V, L>(xk, gk, cs, seg, D, p.eps);
+    store_vec(qo + o1, xq);
+    store_vec(ko + o1, xk);
   }
 }
 

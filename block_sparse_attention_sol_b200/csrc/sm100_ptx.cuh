@@ -93,6 +93,17 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Warp-converged wait for the single-issuer roles (TMA producer, MMA issuer):
+// every lane polls, and the warp agrees on the outcome.  Keeping those warps
+// converged lets the compiler hold descriptors and coordinates in uniform
+// registers; one lane then issues the TMA / MMA / commit instructions.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                               unsigned site, uint64_t limit_ns = SOL_WAIT_LIMIT_NS,
+                                               bool honor_abort = true) {
+  const bool ok = mbar_wait(bar, parity, abort_flag, site, limit_ns, honor_abort);
+  return __all_sync(0xffffffffu, ok);
+}
+
 // ------------------------------------------------------------------ TMA
 // 4-D tiled bulk tensor load into this CTA's shared memory, completing on `bar`.
 __device__ __forceinline__ void tma_load_4d(void* smem_dst, const void* tmap, uint64_t* bar, int c0, int c1, int c2,
@@ -203,6 +214,16 @@ __device__ __forceinline__ void tmem_ld32_wait(uint32_t taddr, uint32_t (&r)[32]
       : "memory");
 }
 
+// 64 consecutive columns of this warp's 32 lanes, then wait: the results are valid when this returns.
+__device__ __forceinline__ void tmem_ld64_wait(uint32_t taddr, uint32_t (&r)[64]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+      : "r"(taddr)
+      : "memory");
+}
+
 // 128 consecutive columns of this warp's 32 lanes, then wait: the results are valid when this returns.
 __device__ __forceinline__ void tmem_ld128_wait(uint32_t taddr, uint32_t (&r)[128]) {
   asm volatile(
@@ -240,6 +261,79 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+
+
+// Packed fp32 pair arithmetic (sm_100): one instruction for two lanes of math.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+
+// 2^x for a pair of fp32 values on the FMA pipe, for x <= 8 (larger inputs
+// are not produced by the attention softmax).  x = n + f with n = floor(x) and
+// f in [0, 1); 2^f comes from a degree-3 polynomial with p(0) = 1 and maximum
+// relative error 8.6e-5 on [0, 1] (minimax fit, csrc/fit_exp2_poly.py); 2^n is
+// added to the exponent field.  Inputs below -127 (including -inf) give 0.
+constexpr float kExp2C1 = 0x1.63e654p-1f;
+constexpr float kExp2C2 = 0x1.d23788p-3f;
+constexpr float kExp2C3 = 0x1.3baadcp-4f;
+__device__ __forceinline__ void exp2_poly_pair(float x0, float x1, float& r0, float& r1) {
+  const float kRound = 12582912.0f;                     // 1.5 * 2^23: adding it exposes floor(x) in the low bits
+  const uint64_t xc = f2_pack(fmaxf(x0, -127.0f), fmaxf(x1, -127.0f));
+  const uint64_t c2 = f2_pack(kRound, kRound);
+  uint64_t t, nf, fr;
+  asm("add.rm.f32x2 %0, %1, %2;" : "=l"(t) : "l"(xc), "l"(c2));       // kRound + floor(x), exactly
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(nf) : "l"(t), "l"(c2));       // floor(x)
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(fr) : "l"(xc), "l"(nf));      // f = x - floor(x), exact
+  uint64_t p = f2_fma(fr, f2_pack(kExp2C3, kExp2C3), f2_pack(kExp2C2, kExp2C2));
+  p = f2_fma(p, fr, f2_pack(kExp2C1, kExp2C1));
+  p = f2_fma(p, fr, f2_pack(1.0f, 1.0f));
+  float t0, t1, p0, p1;
+  f2_unpack(t, t0, t1);
+  f2_unpack(p, p0, p1);
+  const int n0 = __float_as_int(t0) - 0x4B400000;      // bits(kRound + n) - bits(kRound) = n
+  const int n1 = __float_as_int(t1) - 0x4B400000;
+  r0 = __int_as_float(__float_as_int(p0) + (n0 << 23));
+  r1 = __int_as_float(__float_as_int(p1) + (n1 << 23));
+}
+
+
+// Warpgroup register reallocation: every thread of the warpgroup executes it.
+// The increases of all warpgroups must fit in what the decreases free plus the
+// registers the block was launched with.
+template <uint32_t kRegs>
+__device__ __forceinline__ void warpgroup_regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegs));
+}
+template <uint32_t kRegs>
+__device__ __forceinline__ void warpgroup_regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegs));
 }
 
 }  // namespace sol

@@ -133,14 +133,15 @@ sol_status sol_qk_prologue(const void* q_raw, const void* k_raw, void* q_out, vo
     return SOL_ERR_INVALID_ARG;
   if (s.D != 64 && s.D != 128) return SOL_ERR_UNSUPPORTED;
 
+  if (static_cast<long long>(s.B) * s.N >= (1ll << 31)) return SOL_ERR_UNSUPPORTED;
   sol::prologue::Params p;
   p.q_in = q_raw; p.k_in = k_raw; p.q_out = q_out; p.k_out = k_out;
   p.gamma_q = gamma_q; p.gamma_k = gamma_k;
-  p.rows = static_cast<long long>(s.B) * s.N * s.H;
+  p.tokens = s.B * s.N;
   p.N = s.N; p.H = s.H;
   p.gt = s.grid_t; p.gh = s.grid_h; p.gw = s.grid_w;
   p.dt = rope_dt; p.dh = rope_dh; p.dw = rope_dw;
-  p.log2_theta = std::log2(rope_theta);
+  p.log2_theta = std::log2(static_cast<double>(rope_theta));
   p.eps = eps;
   p.tab_t = s.grid_t * (rope_dt / 2);
   p.tab_h = p.tab_t + s.grid_h * (rope_dh / 2);
@@ -150,10 +151,19 @@ sol_status sol_qk_prologue(const void* q_raw, const void* k_raw, void* q_out, vo
 
   DeviceInfo* di = nullptr;
   if (sol_status st = device_info(&di)) return st;
+  // Every row group keeps one head: the number of groups must be a multiple of H.
   const int threads = 256;
   const int lanes_per_row = (dt == SOL_BF16) ? s.D / 8 : s.D / 4;
-  const long long groups_needed = (p.rows + 0) * lanes_per_row / threads + 1;
-  const int grid = static_cast<int>(std::min<long long>(groups_needed, 8ll * di->sm_count));
+  const int groups_per_cta = threads / lanes_per_row;
+  int a = s.H, b = groups_per_cta;
+  while (b) { const int r = a % b; a = b; b = r; }
+  const long long unit = s.H / a;                       // CTAs per whole set of heads
+  const long long needed = (static_cast<long long>(p.tokens) * s.H + groups_per_cta - 1) / groups_per_cta;
+  const long long target = static_cast<long long>(dt == SOL_BF16 ? 3 : 4) * di->sm_count;   // one resident wave
+  long long grid_ll = std::min(needed, target);
+  grid_ll = (grid_ll + unit - 1) / unit * unit;
+  if (grid_ll > 0x7fffffffll) return SOL_ERR_UNSUPPORTED;
+  const int grid = static_cast<int>(grid_ll);
   if (dt == SOL_BF16) {
     if (s.D == 128) sol::prologue::qk_prologue_kernel<__nv_bfloat16, 128><<<grid, threads, smem, stream>>>(p);
     else sol::prologue::qk_prologue_kernel<__nv_bfloat16, 64><<<grid, threads, smem, stream>>>(p);
@@ -260,8 +270,7 @@ sol_status sol_sparse_attn_fwd(const void* q, const void* k, const void* v, cons
   if (s.D != sol::attn100::kHeadDim || block != sol::attn100::kBlock) return SOL_ERR_UNSUPPORTED;
   const long long tiles = static_cast<long long>(s.B) * s.H * nb;
   if (tiles > 0x7fffffffll) return SOL_ERR_UNSUPPORTED;
-  CUtensorMap tq, tk, tv;
-  if (sol_status st = make_bshd_map(&tq, q, s)) return st;
+  CUtensorMap tk, tv;
   if (sol_status st = make_bshd_map(&tk, k, s)) return st;
   if (sol_status st = make_bshd_map(&tv, v, s)) return st;
   const size_t smem = sizeof(sol::attn100::Smem) + 1024;
@@ -272,6 +281,7 @@ sol_status sol_sparse_attn_fwd(const void* q, const void* k, const void* v, cons
     di->attn_attr = true;
   }
   sol::attn100::Params p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
   p.idx = idx;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
@@ -279,7 +289,7 @@ sol_status sol_sparse_attn_fwd(const void* q, const void* k, const void* v, cons
   p.num_tiles = static_cast<int>(tiles);
   p.scale_log2 = scale * 1.4426950408889634f;
   const int grid = static_cast<int>(std::min<long long>(tiles, di->sm_count));
-  sol::attn100::sparse_attn_fwd_kernel<<<grid, sol::attn100::kThreads, smem, stream>>>(tq, tk, tv, p);
+  sol::attn100::sparse_attn_fwd_kernel<<<grid, sol::attn100::kThreads, smem, stream>>>(tk, tv, p);
   return launch_status();
 }
 

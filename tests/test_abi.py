@@ -15,8 +15,11 @@ LIB = os.path.join(ROOT, "block_sparse_attention_sol_b200", "libsol.so")
 @pytest.fixture(scope="module")
 def lib():
     if not os.path.exists(LIB):
-        from block_sparse_attention_sol_b200.build import build
-        build()
+        import importlib.util
+        spec = importlib.util.spec_from_file_location("sol_build", os.path.join(os.path.dirname(LIB), "build.py"))
+        mod = importlib.util.module_from_spec(spec)
+        spec.loader.exec_module(mod)
+        mod.build()
     return ctypes.CDLL(LIB)
 
 
