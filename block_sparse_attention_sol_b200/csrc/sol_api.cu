@@ -293,6 +293,43 @@ sol_status sol_sparse_attn_fwd(const void* q, const void* k, const void* v, cons
   return launch_status();
 }
 
+// ---------------------------------------------------------------- no-alloc select
+// Scratch for sol_block_select_noalloc: one array per device, shared by every
+// call on that device (see include/sol.h for the size limit and the race rule).
+static __device__ __align__(256) unsigned char g_noalloc_scratch[SOL_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+void* g_noalloc_ptr[kMaxDevices] = {};
+std::mutex g_noalloc_mu;
+
+// Host code may not pass g_noalloc_scratch itself to a kernel (on the host it
+// names a stand-in, not device memory): look up its device address once per
+// device, with that device current.
+sol_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SOL_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return SOL_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return SOL_OK;
+}
+}  // namespace
+
+sol_status sol_block_select_noalloc(const void* q, const void* k, sol_shape s, int block, int topk, sol_dtype dt,
+                                    int32_t* idx_out, float* scores_out, cudaStream_t stream) {
+  const size_t need = sol_block_select_workspace_bytes(s, block);
+  if (need == 0) return SOL_ERR_INVALID_ARG;
+  if (need > SOL_NOALLOC_SCRATCH_BYTES) return SOL_ERR_UNSUPPORTED;
+  void* scratch = nullptr;
+  if (sol_status st = noalloc_scratch(&scratch)) return st;
+  return sol_block_select(q, k, s, block, topk, dt, idx_out, scores_out, scratch, SOL_NOALLOC_SCRATCH_BYTES,
+                          stream);
+}
+
 sol_status sol_check_device_status(cudaStream_t stream) {
   if (cudaStreamSynchronize(stream) != cudaSuccess) return SOL_ERR_CUDA;
   unsigned int word = 0;

@@ -120,6 +120,38 @@ sol_status sol_sparse_attn_fwd(const void* q, const void* k, const void* v, cons
                                sol_shape s, int block, int topk, float softmax_scale,
                                sol_dtype dt, void* o, float* lse, cudaStream_t stream);
 
+/*
+ * sol_block_select_noalloc -- sol_block_select for callers that cannot
+ * allocate device memory.  No counterpart on the pages: this is a convenience
+ * of this library.
+ *
+ * Some callers cannot call cudaMalloc: code running inside a host framework's
+ * launch callback or plugin hook that owns all device memory and forbids
+ * allocation there, and latency-critical loops where an allocation (which may
+ * synchronise the device) is not acceptable.  This entry point takes the same
+ * inputs and outputs as sol_block_select but needs no workspace: its scratch
+ * (the pooled means of Q and K) lives in one file-scope device array of
+ * SOL_NOALLOC_SCRATCH_BYTES inside libsol, which every GPU that loads the
+ * library holds until the process exits.
+ *  - Size limit: shapes whose sol_block_select_workspace_bytes() exceeds
+ *    SOL_NOALLOC_SCRATCH_BYTES are rejected with SOL_ERR_UNSUPPORTED before
+ *    anything is launched (the five video workloads need at most 33.4 MB).
+ *  - First call per device: it looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current and caches it; make
+ *    that first call before any stream capture.  A failed lookup returns
+ *    SOL_ERR_CUDA.
+ *  - Sharing: every call on a device uses the same array and it keeps the
+ *    last call's contents.  Nothing in it needs to start at zero (the pooling
+ *    kernel overwrites every byte it later reads), but calls that overlap on
+ *    the GPU (different streams, or different host threads) race on it:
+ *    serialise them.
+ *  - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ */
+#define SOL_NOALLOC_SCRATCH_BYTES (40u * 1024u * 1024u)
+sol_status sol_block_select_noalloc(const void* q, const void* k, sol_shape s, int block, int topk,
+                                    sol_dtype dt, int32_t* idx_out, float* scores_out,
+                                    cudaStream_t stream);
+
 /* Synchronises `stream`, then reads and clears the device error word.
  * Returns SOL_ERR_TIMEOUT if a bounded device wait ran out since the last
  * check, SOL_ERR_CUDA if the stream reports a CUDA error, else SOL_OK. */
