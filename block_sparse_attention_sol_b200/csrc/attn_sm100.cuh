@@ -17,12 +17,15 @@
 //               Keeping Q in TMEM halves the shared-memory operand traffic of the
 //               S MMAs, which would otherwise saturate the tensor core's 128 B/clk
 //               shared-memory read path at N = 128.
-//   warps 2..5  softmax + epilogue: one thread per query row (its TMEM lane).
-//               Each tile starts by loading the thread's Q row from global
-//               memory into TMEM.  Online softmax in the exp2 domain with a lazy
-//               rescale (O is rescaled only when the running max grows by more
-//               than 2^8); P is written to TMEM as bf16 once PV of the previous
-//               step has completed (single P buffer); epilogue O / l -> bf16, LSE.
+//   warps 2..9  softmax + epilogue, two warps per SM sub-partition: each warp
+//               owns 16 TMEM lanes (query rows) and each thread two rows, a
+//               quarter of the columns of each (the .16x256b layout), so one
+//               warp's max/exp work overlaps the other's latency.  Each tile
+//               starts by loading the Q rows from global memory into TMEM.
+//               Online softmax in the exp2 domain with a lazy rescale (O is
+//               rescaled only when the running max grows by more than 2^8); P
+//               is written to TMEM as bf16 once PV of the previous step has
+//               completed (single P buffer); epilogue O / l -> bf16, LSE.
 // TMEM columns: S0 [0,128) S1 [128,256) O [256,384) P [384,448) Q [448,512).
 // Shared memory: K 3 x 32 KB, V 3 x 32 KB.
 //
@@ -39,26 +42,26 @@ namespace attn100 {
 
 constexpr int kBlock = 128;            // tokens per query / key block
 constexpr int kHeadDim = 128;
-constexpr int kKStages = 3;
-constexpr int kVStages = 3;
+constexpr int kSlots = 3;               // K/V ring: slot s holds K_s and V_{s-2} of a tile
 constexpr int kTileBytes = kBlock * kHeadDim * 2;   // 32 KB bf16 tile
 constexpr int kHalfBytes = kTileBytes / 2;          // one 64-column swizzled box
-constexpr int kThreads = 192;
+constexpr int kSoftmaxWarps = 8;
+constexpr int kThreads = 64 + 32 * kSoftmaxWarps;   // producer, MMA, 8 softmax warps
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColO = 256, kColP = 384, kColQ = 448;
 constexpr float kRescaleLog2 = 8.0f;   // lazy-rescale threshold (log2 units)
-// Of every 8 exponential pairs, this many run as a polynomial on the FMA pipe
+// Of every 8 exponentials, this many run as a polynomial on the FMA pipe
 // instead of on MUFU (16 results per clock per SM).
-constexpr int kPolyPairsPer8 = 0;
+constexpr int kPolyPer8 = 0;
 
 struct __align__(1024) Smem {
-  uint8_t k[kKStages][kTileBytes];
-  uint8_t v[kVStages][kTileBytes];
+  uint8_t k[kSlots][kTileBytes];
+  uint8_t v[kSlots][kTileBytes];
   uint64_t q_full, q_empty;
-  uint64_t k_full[kKStages], k_empty[kKStages];
-  uint64_t v_full[kVStages], v_empty[kVStages];
-  uint64_t s_full[2], p_full;
-  uint64_t pv_done, o_free, drain;
+  uint64_t kv_full[kSlots];     // the slot's K and/or V tile has landed
+  uint64_t slot_done[kSlots];   // every MMA reading the slot is complete (for a K slot: S_s readable)
+  uint64_t pv_done;             // PV of the step complete: P writable, O updated
+  uint64_t p_full, o_free, drain;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -74,8 +77,8 @@ struct Params {
 };
 
 // Wait-site ids reported in the error info word.
-enum : unsigned { kSiteQEmpty = 1, kSiteKEmpty, kSiteVEmpty, kSiteQFull, kSiteKFull, kSiteVFull, kSitePFull,
-                  kSiteOFree, kSiteSFull, kSitePvDone, kSiteDrain, kSiteTail };
+enum : unsigned { kSiteQEmpty = 1, kSiteSlotFree, kSiteQFull, kSiteSlotFull, kSitePFull, kSiteOFree, kSiteSDone,
+                  kSitePvDone, kSiteDrain, kSiteTail };
 
 // K-step offsets (16-byte units) inside a 128-byte-swizzled K-major tile: 16
 // channels = 32 bytes per step, the second 64-channel box 16 KB further.
@@ -101,15 +104,12 @@ sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
 
   if (threadIdx.x == 0) {
     sm.abort_flag = 0;
-    mbar_init(&sm.q_full, 4);            // one arrival per softmax warp
+    mbar_init(&sm.q_full, kSoftmaxWarps);   // one arrival per softmax warp
     mbar_init(&sm.q_empty, 1);
-    for (int s = 0; s < kKStages; ++s) { mbar_init(&sm.k_full[s], 1); mbar_init(&sm.k_empty[s], 1); }
-    for (int s = 0; s < kVStages; ++s) { mbar_init(&sm.v_full[s], 1); mbar_init(&sm.v_empty[s], 1); }
-    mbar_init(&sm.s_full[0], 1);
-    mbar_init(&sm.s_full[1], 1);
-    mbar_init(&sm.p_full, 4);
+    for (int s = 0; s < kSlots; ++s) { mbar_init(&sm.kv_full[s], 1); mbar_init(&sm.slot_done[s], 1); }
     mbar_init(&sm.pv_done, 1);
-    mbar_init(&sm.o_free, 4);
+    mbar_init(&sm.p_full, kSoftmaxWarps);
+    mbar_init(&sm.o_free, kSoftmaxWarps);
     mbar_init(&sm.drain, 1);
     fence_mbar_init();
   }
@@ -127,96 +127,94 @@ sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
     if (lane == 0) {
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      uint32_t kq = 0, vq = 0;   // K / V loads issued so far
+      uint32_t sq = 0;   // slots filled so far
       bool ok = true;
       for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
         int b, h, qb;
         decode_tile(p, t, b, h, qb);
         const int32_t* list = p.idx + (static_cast<size_t>(b * p.H + h) * p.nb + qb) * p.topk;
-        // order: K0, K1, V0, K2, V1, ..., V_{k-1}
-        for (int j = 0; j <= p.topk && ok; ++j) {
-          if (j < p.topk) {
-            const int blk = __ldg(list + j);
-            const uint32_t st = kq % kKStages, use = kq / kKStages;
-            if (use > 0 && !(ok = mbar_wait(&sm.k_empty[st], (use - 1) & 1, abort_flag, kSiteKEmpty))) break;
-            mbar_arrive_expect_tx(&sm.k_full[st], kTileBytes);
-            tma_load_4d(sm.k[st], &tm_k, &sm.k_full[st], 0, h, blk * kBlock, b);
-            tma_load_4d(sm.k[st] + kHalfBytes, &tm_k, &sm.k_full[st], 64, h, blk * kBlock, b);
-            ++kq;
+        // slot s of the tile: K_s (s < topk) and V_{s-2} (s >= 2), in the order the MMA issuer uses them
+        for (int s = 0; s < p.topk + 2; ++s, ++sq) {
+          const uint32_t st = sq % kSlots, use = sq / kSlots;
+          if (use > 0 && !(ok = mbar_wait(&sm.slot_done[st], (use - 1) & 1, abort_flag, kSiteSlotFree))) break;
+          const bool has_k = s < p.topk, has_v = s >= 2;
+          mbar_arrive_expect_tx(&sm.kv_full[st], (has_k ? kTileBytes : 0) + (has_v ? kTileBytes : 0));
+          if (has_k) {
+            const int blk = __ldg(list + s);
+            tma_load_4d(sm.k[st], &tm_k, &sm.kv_full[st], 0, h, blk * kBlock, b);
+            tma_load_4d(sm.k[st] + kHalfBytes, &tm_k, &sm.kv_full[st], 64, h, blk * kBlock, b);
           }
-          if (j >= 1) {
-            const int blk = __ldg(list + j - 1);
-            const uint32_t st = vq % kVStages, use = vq / kVStages;
-            if (use > 0 && !(ok = mbar_wait(&sm.v_empty[st], (use - 1) & 1, abort_flag, kSiteVEmpty))) break;
-            mbar_arrive_expect_tx(&sm.v_full[st], kTileBytes);
-            tma_load_4d(sm.v[st], &tm_v, &sm.v_full[st], 0, h, blk * kBlock, b);
-            tma_load_4d(sm.v[st] + kHalfBytes, &tm_v, &sm.v_full[st], 64, h, blk * kBlock, b);
-            ++vq;
+          if (has_v) {
+            const int blk = __ldg(list + s - 2);
+            tma_load_4d(sm.v[st], &tm_v, &sm.kv_full[st], 0, h, blk * kBlock, b);
+            tma_load_4d(sm.v[st] + kHalfBytes, &tm_v, &sm.kv_full[st], 64, h, blk * kBlock, b);
           }
         }
       }
-      // Before the CTA exits, every load issued must have landed (stage s
-      // received loads s, s + stages, ...; wait for the phase of its last one).
-      for (uint32_t s = 0; s < kKStages; ++s)
-        if (s < kq) {
-          const uint32_t uses = (kq - s + kKStages - 1) / kKStages;
-          mbar_wait(&sm.k_full[s], (uses - 1) & 1, abort_flag, kSiteTail, 200000000ull, false);
-        }
-      for (uint32_t s = 0; s < kVStages; ++s)
-        if (s < vq) {
-          const uint32_t uses = (vq - s + kVStages - 1) / kVStages;
-          mbar_wait(&sm.v_full[s], (uses - 1) & 1, abort_flag, kSiteTail, 200000000ull, false);
+      // Before the CTA exits, every load issued must have landed (slot s was
+      // filled for the fills s, s + 3, ...; wait for the phase of its last one).
+      for (uint32_t st = 0; st < kSlots; ++st)
+        if (st < sq) {
+          const uint32_t uses = (sq - st + kSlots - 1) / kSlots;
+          mbar_wait(&sm.kv_full[st], (uses - 1) & 1, abort_flag, kSiteTail, 200000000ull, false);
         }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // tcgen05.mma issue runs only a couple of instructions ahead of execution,
+    // so the tensor pipe idles whenever this thread waits or does bookkeeping.
+    // Each step therefore has one wait point: P_j ready and slot j + 2 (V_j and
+    // K_{j+2}) landed; then PV_j and S_{j+2} go out back to back.  S runs two
+    // steps ahead of PV, so the softmax of step j + 1 finds S_{j+1} complete.
     if (lane == 0) {
       constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, false);
       constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, true);
       const uint32_t q_tm = tmem + kColQ;
       const uint32_t p_tm = tmem + kColP;
       const uint32_t o_tm = tmem + kColO;
-      uint32_t g = 0;
+      uint32_t g = 0;    // steps (S / PV pairs) before this tile
+      uint32_t sq = 0;   // slots before this tile
       int it = 0;
       bool ok = true;
-      // S(gg) = Q K^T into S[gg % 2]
-      auto issue_s = [&](uint32_t gg) -> bool {
-        const uint32_t st = gg % kKStages;
-        if (!mbar_wait(&sm.k_full[st], (gg / kKStages) & 1, abort_flag, kSiteKFull)) return false;
-        tc_fence_after();
+      // S(gg) = Q K^T into S[gg % 2] from slot stage st.  The buffer was last
+      // read by the softmax of step gg - 2, which arrived on p_full before
+      // PV(gg - 2), and with it S(gg), was issued.
+      auto mma_s = [&](uint32_t gg, uint32_t st) {
         const uint64_t kd = smem_desc_sw128(smem_addr(sm.k[st]), 16, 1024);
         const uint32_t d = tmem + kColS + (gg & 1) * 128;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) mma_ts(d, q_tm + kk * 8, kd + kstep_off(kk), kIdescS, kk > 0 ? 1u : 0u);
-        tc_commit(&sm.k_empty[st]);
-        tc_commit(&sm.s_full[gg & 1]);
-        return true;
       };
       for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x, ++it) {
         if (!(ok = mbar_wait(&sm.q_full, it & 1, abort_flag, kSiteQFull))) break;
-        tc_fence_after();
-        if (!(ok = issue_s(g))) break;
+        // slots 0 and 1 of the tile: K_0 and K_1 (slot 1 is empty when topk = 1)
+        for (int s = 0; s < 2 && ok; ++s) {
+          const uint32_t sl = sq + s, st = sl % kSlots;
+          if (!(ok = mbar_wait(&sm.kv_full[st], (sl / kSlots) & 1, abort_flag, kSiteSlotFull))) break;
+          tc_fence_after();
+          if (s < p.topk) mma_s(g + s, st);
+          tc_commit(&sm.slot_done[st]);
+        }
+        if (!ok) break;
+        if (p.topk <= 2) tc_commit(&sm.q_empty);   // every S MMA of this tile has been issued
         for (int j = 0; j < p.topk; ++j) {
-          const uint32_t gg = g + j;
-          if (j + 1 < p.topk) {
-            if (!(ok = issue_s(gg + 1))) break;
-          } else {
-            tc_commit(&sm.q_empty);   // every S MMA of this tile has been issued
-          }
+          const uint32_t gg = g + j, sl = sq + j + 2, st = sl % kSlots;
           if (!(ok = mbar_wait(&sm.p_full, gg & 1, abort_flag, kSitePFull))) break;
           if (j == 0 && it > 0 && !(ok = mbar_wait(&sm.o_free, (it - 1) & 1, abort_flag, kSiteOFree))) break;
-          const uint32_t vs = gg % kVStages;
-          if (!(ok = mbar_wait(&sm.v_full[vs], (gg / kVStages) & 1, abort_flag, kSiteVFull))) break;
+          if (!(ok = mbar_wait(&sm.kv_full[st], (sl / kSlots) & 1, abort_flag, kSiteSlotFull))) break;
           tc_fence_after();
-          const uint64_t vd = smem_desc_sw128(smem_addr(sm.v[vs]), kHalfBytes, 1024);
+          const uint64_t vd = smem_desc_sw128(smem_addr(sm.v[st]), kHalfBytes, 1024);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)   // 16 keys per step: P columns kk*8.., V rows kk*16.. (2 KB)
             mma_ts(o_tm, p_tm + kk * 8, vd + static_cast<uint32_t>(kk * 128), kIdescPV,
                    (j > 0 || kk > 0) ? 1u : 0u);
-          tc_commit(&sm.v_empty[vs]);
           tc_commit(&sm.pv_done);
+          if (j + 2 < p.topk) mma_s(gg + 2, st);
+          tc_commit(&sm.slot_done[st]);
+          if (j + 3 == p.topk) tc_commit(&sm.q_empty);
         }
         g += p.topk;
+        sq += p.topk + 2;
       }
       // Drain: every MMA issued must complete before TMEM is released.
       tc_commit(&sm.drain);
@@ -224,133 +222,159 @@ sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
-    const int quad = warp & 3;                 // TMEM lane quadrant this warp may access
-    const int row = quad * 32 + lane;          // query row inside the tile
-    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    const uint32_t q_addr = tmem + lane_off + kColQ;
-    const uint32_t p_addr = tmem + lane_off + kColP;
-    const uint32_t o_addr = tmem + lane_off + kColO;
+    // Warp w owns the 16 TMEM lanes quad*32 + half*16 .. +15 of its lane
+    // quadrant (quad = w % 4, the quadrant it may access).  Thread 4r + c holds
+    // rows r and r + 8 of them, columns 8i + 2c and 8i + 2c + 1 of each (the
+    // .16x256b layout), so four threads share a row and a row max costs two
+    // shuffles.  P goes back with the .16x128b layout: column 4i + c of a row
+    // is the bf16 pair of keys 8i + 2c, 8i + 2c + 1, which this thread holds.
+    const int quad = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const int r = lane >> 2, c4 = lane & 3;
+    const int row0 = quad * 32 + half * 16 + r;    // this thread's rows: row0 and row0 + 8
+    const uint32_t lanes16 = static_cast<uint32_t>(quad * 32 + half * 16) << 16;
+    const uint32_t lanes32 = static_cast<uint32_t>(quad * 32) << 16;
     const int tail_valid = p.N - (p.nb - 1) * kBlock;   // valid keys in the last block
-    uint32_t g = 0;
+    const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
+    uint32_t g = 0;    // steps before this tile
+    uint32_t sq = 0;   // K/V slots before this tile (topk + 2 per tile)
     int it = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x, ++it) {
       int b, h, qb;
       decode_tile(p, t, b, h, qb);
       const int32_t* list = p.idx + (static_cast<size_t>(b * p.H + h) * p.nb + qb) * p.topk;
-      const int n = qb * kBlock + row;
-      // ---- Q row into TMEM (A operand of the S MMAs: lane = row, 2 bf16 per column)
+      // ---- Q into TMEM (A operand of the S MMAs: lane = row, 2 bf16 per column).
+      // The two warps of a quadrant write channels [64 half, 64 half + 64) of its 32 rows.
       if (it > 0) {
         ok = mbar_wait(&sm.q_empty, (it - 1) & 1, abort_flag, kSiteQEmpty);   // previous tile's S MMAs done
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         tc_fence_after();
       }
       {
-        uint32_t q0[32], q1[32];
-        if (n < p.N) {
-          const uint4* src =
-              reinterpret_cast<const uint4*>(p.q + ((static_cast<size_t>(b) * p.N + n) * p.H + h) * kHeadDim);
+        const int nq = qb * kBlock + quad * 32 + lane;
+        uint32_t qv[32];
+        if (nq < p.N) {
+          const uint4* src = reinterpret_cast<const uint4*>(
+              p.q + ((static_cast<size_t>(b) * p.N + nq) * p.H + h) * kHeadDim + 64 * half);
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
-            const uint4 w0 = __ldg(src + c), w1 = __ldg(src + 8 + c);
-            q0[4 * c] = w0.x; q0[4 * c + 1] = w0.y; q0[4 * c + 2] = w0.z; q0[4 * c + 3] = w0.w;
-            q1[4 * c] = w1.x; q1[4 * c + 1] = w1.y; q1[4 * c + 2] = w1.z; q1[4 * c + 3] = w1.w;
+            const uint4 w = __ldg(src + c);
+            qv[4 * c] = w.x; qv[4 * c + 1] = w.y; qv[4 * c + 2] = w.z; qv[4 * c + 3] = w.w;
           }
         } else {
 #pragma unroll
-          for (int c = 0; c < 32; ++c) { q0[c] = 0u; q1[c] = 0u; }
+          for (int c = 0; c < 32; ++c) qv[c] = 0u;
         }
-        tmem_st32(q_addr, q0);
-        tmem_st32(q_addr + 32, q1);
+        tmem_st32(tmem + lanes32 + kColQ + 32 * half, qv);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.q_full);
       }
-      float m = -INFINITY;   // running max in log2 units (possibly stale by < 2^8)
-      float l = 0.f;         // running sum of exp2(x - m)
+      float m0 = -INFINITY, m1 = -INFINITY;   // running max per row, log2 units (stale by < 2^8)
+      float l0 = 0.f, l1 = 0.f;               // this thread's part of the running sums
       int blk = __ldg(list);
       for (int j = 0; j < p.topk; ++j) {
         const uint32_t gg = g + j;
         const uint32_t buf = gg & 1;
         const int blk_next = (j + 1 < p.topk) ? __ldg(list + j + 1) : 0;
-        ok = mbar_wait(&sm.s_full[buf], (gg >> 1) & 1, abort_flag, kSiteSFull);
+        const uint32_t sl = sq + j;   // slot of K_j: its slot_done also means S_j is complete
+        ok = mbar_wait(&sm.slot_done[sl % kSlots], (sl / kSlots) & 1, abort_flag, kSiteSDone);
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         tc_fence_after();
-        uint32_t sr[128];
-        tmem_ld128_wait(tmem + lane_off + kColS + buf * 128, sr);
+        uint32_t sr[64];   // row0: sr[4i], sr[4i+1]; row0 + 8: sr[4i+2], sr[4i+3]; keys 8i + 2c4 + {0,1}
+        tmem_ld16x256b_x16_wait(tmem + lanes16 + kColS + buf * 128, sr);
         if (blk == p.nb - 1 && tail_valid < kBlock) {
 #pragma unroll
-          for (int e = 0; e < 128; ++e)
-            if (e >= tail_valid) sr[e] = __float_as_uint(-INFINITY);
+          for (int i = 0; i < 16; ++i)
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              if (8 * i + 2 * c4 + (e & 1) >= tail_valid) sr[4 * i + e] = __float_as_uint(-INFINITY);
         }
-        // row max: 16 independent chains, then a small tree
-        float pm[16];
+        // row max: two chains per row, then across the four threads of the row
+        float pm[4];
 #pragma unroll
-        for (int c = 0; c < 16; ++c) pm[c] = fmaxf(__uint_as_float(sr[c]), __uint_as_float(sr[c + 16]));
+        for (int e = 0; e < 4; ++e) {
+          pm[e] = fmaxf(__uint_as_float(sr[e]), __uint_as_float(sr[4 + e]));
 #pragma unroll
-        for (int e = 32; e < 128; e += 32)
+          for (int i = 2; i < 16; i += 2)
+            pm[e] = fmax3(pm[e], __uint_as_float(sr[4 * i + e]), __uint_as_float(sr[4 * i + 4 + e]));
+        }
+        float mx0 = fmaxf(pm[0], pm[1]), mx1 = fmaxf(pm[2], pm[3]);
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2)) * p.scale_log2;
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2)) * p.scale_log2;
+        const bool rs0 = mx0 > m0 + kRescaleLog2, rs1 = mx1 > m1 + kRescaleLog2;
+        const float mu0 = rs0 ? mx0 : m0, mu1 = rs1 ? mx1 : m1;
+        const uint64_t nm0 = f2_pack(-mu0, -mu0), nm1 = f2_pack(-mu1, -mu1);
+        // P = exp2(s * scale - m) as bf16 pairs; two partial sums per row
+        uint32_t pk[32];
+        uint64_t acc0[2] = {0ull, 0ull}, acc1[2] = {0ull, 0ull};
 #pragma unroll
-          for (int c = 0; c < 16; ++c)
-            pm[c] = fmax3(pm[c], __uint_as_float(sr[e + c]), __uint_as_float(sr[e + 16 + c]));
-#pragma unroll
-        for (int c = 0; c < 5; ++c) pm[c] = fmax3(pm[c], pm[c + 5], pm[c + 10]);
-        const float mx = fmaxf(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[15])) * p.scale_log2;
-        const bool rescale = mx > m + kRescaleLog2;
-        const float m_use = rescale ? mx : m;
-        const uint64_t neg_m2 = f2_pack(-m_use, -m_use);
-        const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
-        // P = exp2(s * scale - m) as bf16 pairs (kept in registers); 8 partial sums
-        uint32_t pk0[32], pk1[32];
-        uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
-#pragma unroll
-        for (int e = 0; e < 128; e += 2) {
-          float a0, a1;
-          f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])), scale2, neg_m2), a0, a1);
-          float p0, p1;
-          if (((e >> 1) & 7) >= 8 - kPolyPairsPer8) {
-            exp2_poly_pair(a0, a1, p0, p1);        // FMA pipe
+        for (int i = 0; i < 16; ++i) {
+          float x0, x1, x2, x3;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[4 * i]), __uint_as_float(sr[4 * i + 1])), scale2, nm0), x0, x1);
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[4 * i + 2]), __uint_as_float(sr[4 * i + 3])), scale2, nm1), x2,
+                    x3);
+          float p0, p1, p2, p3;
+          if ((i & 7) >= 8 - kPolyPer8) {
+            exp2_poly_pair(x0, x1, p0, p1);   // FMA pipe
+            exp2_poly_pair(x2, x3, p2, p3);
           } else {
-            p0 = ex2_approx(a0);                   // MUFU
-            p1 = ex2_approx(a1);
+            p0 = ex2_approx(x0);              // MUFU
+            p1 = ex2_approx(x1);
+            p2 = ex2_approx(x2);
+            p3 = ex2_approx(x3);
           }
-          acc[(e >> 1) & 3] = f2_add(acc[(e >> 1) & 3], f2_pack(p0, p1));
-          if (e < 64) pk0[e >> 1] = pack_bf16x2(p0, p1);
-          else pk1[(e - 64) >> 1] = pack_bf16x2(p0, p1);
+          acc0[i & 1] = f2_add(acc0[i & 1], f2_pack(p0, p1));
+          acc1[i & 1] = f2_add(acc1[i & 1], f2_pack(p2, p3));
+          pk[2 * i] = pack_bf16x2(p0, p1);
+          pk[2 * i + 1] = pack_bf16x2(p2, p3);
         }
-        float rs0, rs1, rs2, rs3;
-        f2_unpack(f2_add(acc[0], acc[1]), rs0, rs1);
-        f2_unpack(f2_add(acc[2], acc[3]), rs2, rs3);
-        const float rowsum = (rs0 + rs1) + (rs2 + rs3);
+        float s0a, s0b, s1a, s1b;
+        f2_unpack(f2_add(acc0[0], acc0[1]), s0a, s0b);
+        f2_unpack(f2_add(acc1[0], acc1[1]), s1a, s1b);
         if (j > 0) {
-          // PV of the previous step must be done before P is overwritten and O
-          // rescaled; waited every step so this thread tracks every phase.
+          // PV of the previous step must be done before P is overwritten and O rescaled.
           ok = mbar_wait(&sm.pv_done, (gg - 1) & 1, abort_flag, kSitePvDone);
           if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
           tc_fence_after();
-          if (__any_sync(0xffffffffu, rescale)) {
-            const float alpha = rescale ? ex2_approx(m - m_use) : 1.f;
-            const uint64_t alpha2 = f2_pack(alpha, alpha);
+        }
+        tmem_st16x128b_x16(tmem + lanes16 + kColP, pk);   // 128 keys -> 64 columns of bf16 pairs
+        // O is rescaled after P is stored (P's registers are free by then) and
+        // before p_full, which is what lets the next PV accumulate into O.
+        if (j > 0) {
+          if (__any_sync(0xffffffffu, rs0 || rs1)) {
+            const float al0 = rs0 ? ex2_approx(m0 - mu0) : 1.f;
+            const float al1 = rs1 ? ex2_approx(m1 - mu1) : 1.f;
+            const uint64_t a0 = f2_pack(al0, al0), a1 = f2_pack(al1, al1);
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
+            for (int hc = 0; hc < 2; ++hc) {   // O columns [64 hc, 64 hc + 64)
               uint32_t orr[32];
-              tmem_ld32_wait(o_addr + c * 32, orr);
+              tmem_ld16x256b_x8_wait(tmem + lanes16 + kColO + 64 * hc, orr);
 #pragma unroll
-              for (int e = 0; e < 32; e += 2) {
-                float o0, o1;
-                f2_unpack(f2_mul(f2_pack(__uint_as_float(orr[e]), __uint_as_float(orr[e + 1])), alpha2), o0, o1);
-                orr[e] = __float_as_uint(o0);
-                orr[e + 1] = __float_as_uint(o1);
+              for (int i = 0; i < 8; ++i) {
+                float o0, o1, o2, o3;
+                f2_unpack(f2_mul(f2_pack(__uint_as_float(orr[4 * i]), __uint_as_float(orr[4 * i + 1])), a0), o0, o1);
+                f2_unpack(f2_mul(f2_pack(__uint_as_float(orr[4 * i + 2]), __uint_as_float(orr[4 * i + 3])), a1), o2,
+                          o3);
+                orr[4 * i] = __float_as_uint(o0);
+                orr[4 * i + 1] = __float_as_uint(o1);
+                orr[4 * i + 2] = __float_as_uint(o2);
+                orr[4 * i + 3] = __float_as_uint(o3);
               }
-              tmem_st32(o_addr + c * 32, orr);
+              tmem_st16x256b_x8(tmem + lanes16 + kColO + 64 * hc, orr);
             }
-            l *= alpha;
+            l0 *= al0;
+            l1 *= al1;
           }
         }
-        tmem_st32(p_addr, pk0);          // 128 keys -> 64 columns of bf16 pairs
-        tmem_st32(p_addr + 32, pk1);
-        m = m_use;
-        l += rowsum;
+        m0 = mu0;
+        m1 = mu1;
+        l0 += s0a + s0b;
+        l1 += s1a + s1b;
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -359,33 +383,49 @@ sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
       }
       if (!ok) break;
       // epilogue: O / l and LSE
-      ok = mbar_wait(&sm.pv_done, (g + p.topk - 1) & 1, abort_flag, kSitePvDone);
+      {
+        ok = mbar_wait(&sm.pv_done, (g + p.topk - 1) & 1, abort_flag, kSitePvDone);
+      }
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
-      uint32_t orr[128];
-      tmem_ld128_wait(o_addr, orr);
+      l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+      l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+      const float inv0 = 1.f / l0, inv1 = 1.f / l1;
+      const uint64_t i0 = f2_pack(inv0, inv0), i1 = f2_pack(inv1, inv1);
+      uint32_t ob[2][16];   // bf16 pairs of O / l: row u, channels 8i + 2c4, 8i + 2c4 + 1
+#pragma unroll
+      for (int hc = 0; hc < 2; ++hc) {
+        uint32_t orr[32];
+        tmem_ld16x256b_x8_wait(tmem + lanes16 + kColO + 64 * hc, orr);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          float o0, o1, o2, o3;
+          f2_unpack(f2_mul(f2_pack(__uint_as_float(orr[4 * i]), __uint_as_float(orr[4 * i + 1])), i0), o0, o1);
+          f2_unpack(f2_mul(f2_pack(__uint_as_float(orr[4 * i + 2]), __uint_as_float(orr[4 * i + 3])), i1), o2, o3);
+          ob[0][8 * hc + i] = pack_bf16x2(o0, o1);
+          ob[1][8 * hc + i] = pack_bf16x2(o2, o3);
+        }
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.o_free);
-      if (n < p.N) {
-        const float inv = 1.f / l;
-        const uint64_t inv2 = f2_pack(inv, inv);
-        uint4* dst = reinterpret_cast<uint4*>(p.o + ((static_cast<size_t>(b) * p.N + n) * p.H + h) * kHeadDim);
+      const int n0 = qb * kBlock + row0;
 #pragma unroll
-        for (int e = 0; e < 128; e += 8) {
-          uint32_t w[4];
+      for (int u = 0; u < 2; ++u) {
+        const int n = n0 + 8 * u;
+        if (n < p.N) {
+          uint32_t* dst = reinterpret_cast<uint32_t*>(p.o + ((static_cast<size_t>(b) * p.N + n) * p.H + h) * kHeadDim);
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            float o0, o1;
-            f2_unpack(f2_mul(f2_pack(__uint_as_float(orr[e + 2 * u]), __uint_as_float(orr[e + 2 * u + 1])), inv2),
-                      o0, o1);
-            w[u] = pack_bf16x2(o0, o1);
-          }
-          dst[e / 8] = make_uint4(w[0], w[1], w[2], w[3]);
+          for (int i = 0; i < 16; ++i) dst[4 * i + c4] = ob[u][i];
+          if (c4 == 0)
+            p.lse[(static_cast<size_t>(b) * p.H + h) * p.N + n] =
+                ((u ? m1 : m0) + __log2f(u ? l1 : l0)) * 0.69314718055994531f;
         }
-        p.lse[(static_cast<size_t>(b) * p.H + h) * p.N + n] = (m + __log2f(l)) * 0.69314718055994531f;
       }
       g += p.topk;
+      sq += p.topk + 2;
     }
   }
 
