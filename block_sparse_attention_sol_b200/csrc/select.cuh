@@ -5,13 +5,16 @@
 //   pool:   qbar[b,h,i,:] = mean of q[b,n,h,:] over the valid tokens n of block i
 //           (same for k).  HBM-bound: one CTA per (b, block, tensor) streams the
 //           block's rows (all heads, contiguous) with 16-byte loads.
-//   score:  s[b,h,i,j] = qbar[b,h,i,:] . kbar[b,h,j,:]  in fp32 (register-tiled
-//           SIMT; a tensor-core score would round the scores and move the top-k
-//           boundary).
+//   score:  s[b,h,i,j] = qbar[b,h,i,:] . kbar[b,h,j,:]  in fp32 (SIMT FMA; a
+//           tensor-core score would round the scores and move the top-k
+//           boundary).  A CTA keeps 32 (or 16) rows' scores in shared memory;
+//           each thread computes 4 rows x 4 keys of a 128-key chunk: 16-byte
+//           shared loads, rows broadcast across the warp, keys 32 apart.
 //   top-k:  per row, the k largest scores, exact ties to the lower j, written in
-//           ascending j.  A warp finds the k-th largest order-preserving key by a
-//           most-significant-bit-first search of the 32-bit key space, then
-//           compacts the winners in ascending j with ballots.
+//           ascending j.  A warp holds the row's order-preserving keys in
+//           registers, finds the k-th largest by a most-significant-bit-first
+//           search of the 32-bit key space, then compacts the winners in
+//           ascending j with ballots.
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -70,24 +73,68 @@ __global__ void __launch_bounds__(256) block_pool_kernel(const T* __restrict__ q
 }
 
 // ------------------------------------------------------------------ scores + top-k
-constexpr int kRows = 16;        // query blocks per CTA
-constexpr int kKeys = 64;        // key blocks per shared-memory chunk
-constexpr int kThreads = 256;
+// A CTA scores 8 * RPW query blocks (RPW rows per warp: 4, or 2 when 32 rows of
+// scores do not fit in shared memory) against all key blocks, in chunks of kKeys.
+constexpr int kKeys = 128;       // key blocks per shared-memory chunk
+constexpr int kThreads = 256;    // warp w: rows RPW w .. +RPW-1; lane l: keys l + {0, 32, 64, 96} of a chunk
+constexpr int kMaxNb = 2048;
+
+__host__ __device__ constexpr size_t score_topk_smem_bytes(int D, int rows, int nb) {
+  return (static_cast<size_t>(D + 4) * (rows + kKeys) + static_cast<size_t>(rows) * nb) * sizeof(float);
+}
 
 __device__ __forceinline__ uint32_t order_key(float f) {
   const uint32_t u = __float_as_uint(f + 0.0f);   // -0 -> +0 so equal scores get equal keys
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Dynamic shared memory: qs[kRows][D+4] | ks[kKeys][D+4] | sc[kRows][nb]
-// grid (ceil(nb / kRows), B * H).
-template <int D>
-__global__ void __launch_bounds__(kThreads) score_topk_kernel(const float* __restrict__ qbar,
-                                                              const float* __restrict__ kbar,
-                                                              int32_t* __restrict__ idx, float* __restrict__ scores_out,
-                                                              int nb, int topk) {
+// The k-th largest key of a row held as KPL keys per lane (key j at lane j % 32,
+// slot j / 32; 0 pads, below every real key), then the row's ids with key above
+// it, plus the first (topk - count above) with key equal to it, in ascending j.
+template <int KPL>
+__device__ __forceinline__ void topk_row(const uint32_t (&key)[KPL], int nb, int topk, int32_t* out, int lane) {
+  uint32_t prefix = 0u;   // largest T with count(key >= T) >= topk, built bit by bit
+#pragma unroll 1
+  for (int bit = 31; bit >= 0; --bit) {
+    const uint32_t cand = prefix | (1u << bit);
+    uint32_t cnt = 0;
+#pragma unroll
+    for (int q = 0; q < KPL; ++q) cnt += key[q] >= cand ? 1u : 0u;
+    if (static_cast<int>(__reduce_add_sync(0xffffffffu, cnt)) >= topk) prefix = cand;
+  }
+  uint32_t gt = 0;
+#pragma unroll
+  for (int q = 0; q < KPL; ++q) gt += key[q] > prefix ? 1u : 0u;
+  const int need_eq = topk - static_cast<int>(__reduce_add_sync(0xffffffffu, gt));
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  int written = 0, eq_seen = 0;
+#pragma unroll
+  for (int q = 0; q < KPL; ++q) {
+    if (q * 32 >= nb) break;
+    const int j = q * 32 + lane;
+    const bool is_gt = key[q] > prefix;
+    const bool is_eq = key[q] == prefix;
+    const uint32_t eq_mask = __ballot_sync(0xffffffffu, is_eq);
+    const int eq_rank = eq_seen + __popc(eq_mask & lt_mask);
+    const bool sel = is_gt || (is_eq && eq_rank < need_eq);
+    const uint32_t sel_mask = __ballot_sync(0xffffffffu, sel);
+    if (sel) out[written + __popc(sel_mask & lt_mask)] = j;
+    written += __popc(sel_mask);
+    eq_seen += __popc(eq_mask);
+  }
+}
+
+// Dynamic shared memory: qs[rows][D+4] | ks[kKeys][D+4] | sc[rows][nb].  The 4-float row
+// padding puts the 16-byte loads of 8 consecutive rows on distinct banks.
+// grid (ceil(nb / (8 RPW)), B * H).  KPL = keys per lane in the top-k, nb <= 32 * KPL.
+template <int D, int RPW, int KPL>
+__global__ void __launch_bounds__(kThreads, 1) score_topk_kernel(const float* __restrict__ qbar,
+                                                                 const float* __restrict__ kbar,
+                                                                 int32_t* __restrict__ idx,
+                                                                 float* __restrict__ scores_out, int nb, int topk) {
   extern __shared__ float smem[];
   constexpr int P = D + 4;
+  constexpr int kRows = 8 * RPW;
   float* qs = smem;
   float* ks = qs + kRows * P;
   float* sc = ks + kKeys * P;
@@ -100,37 +147,49 @@ __global__ void __launch_bounds__(kThreads) score_topk_kernel(const float* __res
   for (int e = threadIdx.x; e < kRows * (D / 4); e += kThreads) {
     const int r = e / (D / 4), d = (e % (D / 4)) * 4;
     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (r < nrows) v = *reinterpret_cast<const float4*>(qb + static_cast<size_t>(r0 + r) * D + d);
+    if (r < nrows) v = __ldg(reinterpret_cast<const float4*>(qb + static_cast<size_t>(r0 + r) * D + d));
     *reinterpret_cast<float4*>(qs + r * P + d) = v;
   }
-  // thread -> (4 rows, 1 key) of a 16 x 64 chunk
-  const int kj = threadIdx.x % kKeys;
-  const int rg = (threadIdx.x / kKeys) * 4;
+  const int lane = threadIdx.x & 31;
+  const int rg = (threadIdx.x >> 5) * RPW;   // this warp's rows
   for (int j0 = 0; j0 < nb; j0 += kKeys) {
-    __syncthreads();
+    __syncthreads();   // previous chunk fully consumed (and qs written, the first time)
     for (int e = threadIdx.x; e < kKeys * (D / 4); e += kThreads) {
       const int j = e / (D / 4), d = (e % (D / 4)) * 4;
       float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (j0 + j < nb) v = *reinterpret_cast<const float4*>(kb + static_cast<size_t>(j0 + j) * D + d);
+      if (j0 + j < nb) v = __ldg(reinterpret_cast<const float4*>(kb + static_cast<size_t>(j0 + j) * D + d));
       *reinterpret_cast<float4*>(ks + j * P + d) = v;
     }
     __syncthreads();
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 8
-    for (int d = 0; d < D; d += 4) {
-      const float4 kv = *reinterpret_cast<const float4*>(ks + kj * P + d);
+    float acc[RPW][4];   // [row][key lane + 32 c]
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const float4 qv = *reinterpret_cast<const float4*>(qs + (rg + r) * P + d);
-        acc[r] = fmaf(qv.x, kv.x, acc[r]);
-        acc[r] = fmaf(qv.y, kv.y, acc[r]);
-        acc[r] = fmaf(qv.z, kv.z, acc[r]);
-        acc[r] = fmaf(qv.w, kv.w, acc[r]);
-      }
+    for (int r = 0; r < RPW; ++r)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[r][c] = 0.f;
+#pragma unroll 4
+    for (int d = 0; d < D; d += 4) {   // channels in ascending order: one fixed fp32 rounding sequence per score
+      float4 qv[RPW], kv[4];
+#pragma unroll
+      for (int r = 0; r < RPW; ++r) qv[r] = *reinterpret_cast<const float4*>(qs + (rg + r) * P + d);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) kv[c] = *reinterpret_cast<const float4*>(ks + (lane + 32 * c) * P + d);
+#pragma unroll
+      for (int r = 0; r < RPW; ++r)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          acc[r][c] = fmaf(qv[r].x, kv[c].x, acc[r][c]);
+          acc[r][c] = fmaf(qv[r].y, kv[c].y, acc[r][c]);
+          acc[r][c] = fmaf(qv[r].z, kv[c].z, acc[r][c]);
+          acc[r][c] = fmaf(qv[r].w, kv[c].w, acc[r][c]);
+        }
     }
-    if (j0 + kj < nb) {
 #pragma unroll
-      for (int r = 0; r < 4; ++r) sc[(rg + r) * nb + j0 + kj] = acc[r];
+    for (int c = 0; c < 4; ++c) {
+      const int j = j0 + lane + 32 * c;
+      if (j < nb) {
+#pragma unroll
+        for (int r = 0; r < RPW; ++r) sc[(rg + r) * nb + j] = acc[r][c];
+      }
     }
   }
   __syncthreads();
@@ -142,45 +201,16 @@ __global__ void __launch_bounds__(kThreads) score_topk_kernel(const float* __res
     }
   }
 
-  __syncthreads();   // the dump above reads rows the key conversion below rewrites
-
-  // top-k: one warp per row
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t lt_mask = (1u << lane) - 1u;
+  // top-k: one warp per row, the row's keys in registers
+  const int warp = threadIdx.x >> 5;
   for (int r = warp; r < nrows; r += kThreads / 32) {
-    uint32_t* keys = reinterpret_cast<uint32_t*>(sc + r * nb);
-    for (int j = lane; j < nb; j += 32) keys[j] = order_key(sc[r * nb + j]);
-    __syncwarp();
-    // largest T with count(key >= T) >= topk, i.e. the k-th largest key
-    uint32_t prefix = 0u;
-    for (int bit = 31; bit >= 0; --bit) {
-      const uint32_t cand = prefix | (1u << bit);
-      int cnt = 0;
-      for (int j = lane; j < nb; j += 32) cnt += keys[j] >= cand ? 1 : 0;
+    uint32_t key[KPL];
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
-      if (cnt >= topk) prefix = cand;
+    for (int q = 0; q < KPL; ++q) {
+      const int j = q * 32 + lane;
+      key[q] = j < nb ? order_key(sc[r * nb + j]) : 0u;
     }
-    int gt = 0;
-    for (int j = lane; j < nb; j += 32) gt += keys[j] > prefix ? 1 : 0;
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) gt += __shfl_xor_sync(0xffffffffu, gt, off);
-    const int need_eq = topk - gt;
-    int32_t* out = idx + (static_cast<size_t>(bh) * nb + r0 + r) * topk;
-    int written = 0, eq_seen = 0;
-    for (int j0 = 0; j0 < nb; j0 += 32) {
-      const int j = j0 + lane;
-      const uint32_t key = j < nb ? keys[j] : 0u;
-      const bool is_gt = j < nb && key > prefix;
-      const bool is_eq = j < nb && key == prefix;
-      const uint32_t eq_mask = __ballot_sync(0xffffffffu, is_eq);
-      const int eq_rank = eq_seen + __popc(eq_mask & lt_mask);
-      const bool sel = is_gt || (is_eq && eq_rank < need_eq);
-      const uint32_t sel_mask = __ballot_sync(0xffffffffu, sel);
-      if (sel) out[written + __popc(sel_mask & lt_mask)] = j;
-      written += __popc(sel_mask);
-      eq_seen += __popc(eq_mask);
-    }
+    topk_row<KPL>(key, nb, topk, idx + (static_cast<size_t>(bh) * nb + r0 + r) * topk, lane);
   }
 }
 

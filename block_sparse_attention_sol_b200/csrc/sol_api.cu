@@ -25,6 +25,7 @@
 namespace {
 
 constexpr int kMaxDevices = 64;
+constexpr size_t kMaxSmemPerBlock = 227 * 1024;   // opt-in dynamic shared memory per CTA on sm_100
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -42,7 +43,8 @@ int num_blocks(int N, int block) { return (N + block - 1) / block; }
 
 struct DeviceInfo {
   int sm_count = 0;
-  bool attn_attr = false, select_attr64 = false, select_attr128 = false;
+  bool attn_attr = false;
+  bool select_attr[16] = {};   // score_topk_kernel instantiations with the shared-memory opt-in set
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -103,6 +105,47 @@ __global__ void wait_timeout_selftest_kernel(unsigned long long limit_ns) {
     // nothing ever arrives on `bar`: the bounded wait must give up and report
     sol::mbar_wait(&bar, 0, &abort_flag, 0xFFu, limit_ns);
   }
+}
+
+}  // namespace
+
+namespace {
+
+// Launches score_topk_kernel<D, RPW, KPL> for the runtime choices (shared-memory
+// opt-in set once per device and instantiation).
+template <int D, int RPW, int KPL>
+sol_status launch_score_topk_t(DeviceInfo* di, dim3 grid, size_t smem, cudaStream_t stream, const float* qbar,
+                               const float* kbar, int32_t* idx, float* scores, int nb, int topk) {
+  constexpr int slot = (D == 128 ? 8 : 0) + (RPW == 4 ? 4 : 0) + (KPL == 8 ? 0 : KPL == 16 ? 1 : KPL == 32 ? 2 : 3);
+  if (!di->select_attr[slot]) {
+    if (cudaFuncSetAttribute(sol::select::score_topk_kernel<D, RPW, KPL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kMaxSmemPerBlock)) != cudaSuccess)
+      return SOL_ERR_CUDA;
+    di->select_attr[slot] = true;
+  }
+  sol::select::score_topk_kernel<D, RPW, KPL><<<grid, sol::select::kThreads, smem, stream>>>(qbar, kbar, idx, scores,
+                                                                                            nb, topk);
+  return launch_status();
+}
+
+template <int D, int RPW>
+sol_status launch_score_topk_k(DeviceInfo* di, int kpl, dim3 grid, size_t smem, cudaStream_t stream,
+                               const float* qbar, const float* kbar, int32_t* idx, float* scores, int nb, int topk) {
+  switch (kpl) {
+    case 8: return launch_score_topk_t<D, RPW, 8>(di, grid, smem, stream, qbar, kbar, idx, scores, nb, topk);
+    case 16: return launch_score_topk_t<D, RPW, 16>(di, grid, smem, stream, qbar, kbar, idx, scores, nb, topk);
+    case 32: return launch_score_topk_t<D, RPW, 32>(di, grid, smem, stream, qbar, kbar, idx, scores, nb, topk);
+    default: return launch_score_topk_t<D, RPW, 64>(di, grid, smem, stream, qbar, kbar, idx, scores, nb, topk);
+  }
+}
+
+sol_status launch_score_topk(DeviceInfo* di, int D, int rpw, int kpl, dim3 grid, size_t smem, cudaStream_t stream,
+                             const float* qbar, const float* kbar, int32_t* idx, float* scores, int nb, int topk) {
+  if (D == 128)
+    return rpw == 4 ? launch_score_topk_k<128, 4>(di, kpl, grid, smem, stream, qbar, kbar, idx, scores, nb, topk)
+                    : launch_score_topk_k<128, 2>(di, kpl, grid, smem, stream, qbar, kbar, idx, scores, nb, topk);
+  return rpw == 4 ? launch_score_topk_k<64, 4>(di, kpl, grid, smem, stream, qbar, kbar, idx, scores, nb, topk)
+                  : launch_score_topk_k<64, 2>(di, kpl, grid, smem, stream, qbar, kbar, idx, scores, nb, topk);
 }
 
 }  // namespace
@@ -174,6 +217,7 @@ sol_status sol_qk_prologue(const void* q_raw, const void* k_raw, void* q_out, vo
   return launch_status();
 }
 
+
 size_t sol_block_select_workspace_bytes(sol_shape s, int block) {
   if (!shape_ok(s) || block <= 0) return 0;
   return 2ull * s.B * s.H * static_cast<size_t>(num_blocks(s.N, block)) * s.D * sizeof(float);
@@ -209,29 +253,13 @@ sol_status sol_block_select(const void* q, const void* k, sol_shape s, int block
                                                                   s.D, block, nb);
   if (sol_status st = launch_status()) return st;
 
-  const size_t smem = (static_cast<size_t>(sol::select::kRows + sol::select::kKeys) * (s.D + 4) +
-                       static_cast<size_t>(sol::select::kRows) * nb) * sizeof(float);
-  dim3 sg((nb + sol::select::kRows - 1) / sol::select::kRows, s.B * s.H);
-  if (s.D == 128) {
-    if (!di->select_attr128) {
-      if (cudaFuncSetAttribute(sol::select::score_topk_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               200 * 1024) != cudaSuccess)
-        return SOL_ERR_CUDA;
-      di->select_attr128 = true;
-    }
-    sol::select::score_topk_kernel<128><<<sg, sol::select::kThreads, smem, stream>>>(qbar, kbar, idx_out, scores_out,
-                                                                                     nb, topk);
-  } else {
-    if (!di->select_attr64) {
-      if (cudaFuncSetAttribute(sol::select::score_topk_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               200 * 1024) != cudaSuccess)
-        return SOL_ERR_CUDA;
-      di->select_attr64 = true;
-    }
-    sol::select::score_topk_kernel<64><<<sg, sol::select::kThreads, smem, stream>>>(qbar, kbar, idx_out, scores_out,
-                                                                                    nb, topk);
-  }
-  return launch_status();
+  // 32 rows per CTA when their scores fit in shared memory, else 16.
+  const int rpw = sol::select::score_topk_smem_bytes(s.D, 32, nb) <= kMaxSmemPerBlock ? 4 : 2;
+  const size_t smem = sol::select::score_topk_smem_bytes(s.D, 8 * rpw, nb);
+  if (smem > kMaxSmemPerBlock) return SOL_ERR_UNSUPPORTED;
+  const int kpl = nb <= 256 ? 8 : nb <= 512 ? 16 : nb <= 1024 ? 32 : 64;
+  const dim3 sg((nb + 8 * rpw - 1) / (8 * rpw), s.B * s.H);
+  return launch_score_topk(di, s.D, rpw, kpl, sg, smem, stream, qbar, kbar, idx_out, scores_out, nb, topk);
 }
 
 sol_status sol_sparse_attn_fwd(const void* q, const void* k, const void* v, const int32_t* idx, sol_shape s,
