@@ -23,6 +23,7 @@ import torch
 __all__ = [
     "SolError", "SolShape", "LIB_PATH", "lib",
     "sol_qk_prologue", "sol_block_select", "sol_block_select_workspace_bytes", "sol_sparse_attn_fwd",
+    "sol_qk_prologue_pool", "sol_block_select_pooled",
     "sol_check_device_status", "sol_selftest_wait_timeout", "sol_status_string", "sol_attention_chain",
     "SOL_OK", "SOL_ERR_INVALID_ARG", "SOL_ERR_UNSUPPORTED", "SOL_ERR_CUDA", "SOL_ERR_TIMEOUT",
 ]
@@ -57,6 +58,10 @@ lib.sol_block_select_workspace_bytes.restype = _SZ
 lib.sol_block_select_workspace_bytes.argtypes = [SolShape, _I]
 lib.sol_block_select.restype = _I
 lib.sol_block_select.argtypes = [_P, _P, SolShape, _I, _I, _I, _P, _P, _P, _SZ, _P]
+lib.sol_qk_prologue_pool.restype = _I
+lib.sol_qk_prologue_pool.argtypes = [_P, _P, _P, _P, _P, _P, SolShape, _I, _I, _I, _F, _F, _I, _I, _P, _P, _P]
+lib.sol_block_select_pooled.restype = _I
+lib.sol_block_select_pooled.argtypes = [_P, _P, SolShape, _I, _I, _P, _P, _P]
 lib.sol_sparse_attn_fwd.restype = _I
 lib.sol_sparse_attn_fwd.argtypes = [_P, _P, _P, _P, SolShape, _I, _I, _F, _I, _P, _P, _P]
 lib.sol_check_device_status.restype = _I
@@ -118,6 +123,49 @@ def sol_qk_prologue(q_raw, k_raw, gamma_q, gamma_k, grid, rope_split=None, rope_
                              _stream_handle(stream))
     _check(st, "sol_qk_prologue")
     return q_out, k_out
+
+
+def sol_qk_prologue_pool(q_raw, k_raw, gamma_q, gamma_k, grid, block, rope_split=None, rope_theta=10000.0,
+                         eps=1e-6, q_out=None, k_out=None, qbar_out=None, kbar_out=None, stream=None):
+    """sol_qk_prologue plus the fp32 block means of its stored outputs.
+    Returns (q, k, qbar, kbar); qbar, kbar are [B, H, nb, D]."""
+    _cuda(q_raw, "q_raw"), _cuda(k_raw, "k_raw"), _cuda(gamma_q, "gamma_q"), _cuda(gamma_k, "gamma_k")
+    s = _shape(q_raw, grid)
+    if rope_split is None:
+        dh = 2 * (s.D // 6)
+        rope_split = (s.D - 2 * dh, dh, dh)
+    nb = -(-s.N // block)
+    q_out = torch.empty_like(q_raw) if q_out is None else _cuda(q_out, "q_out")
+    k_out = torch.empty_like(k_raw) if k_out is None else _cuda(k_out, "k_out")
+    pooled = (s.B, s.H, nb, s.D)
+    qbar_out = (torch.empty(pooled, dtype=torch.float32, device=q_raw.device) if qbar_out is None
+                else _cuda(qbar_out, "qbar_out"))
+    kbar_out = (torch.empty(pooled, dtype=torch.float32, device=q_raw.device) if kbar_out is None
+                else _cuda(kbar_out, "kbar_out"))
+    st = lib.sol_qk_prologue_pool(q_raw.data_ptr(), k_raw.data_ptr(), q_out.data_ptr(), k_out.data_ptr(),
+                                  gamma_q.data_ptr(), gamma_k.data_ptr(), s, int(rope_split[0]), int(rope_split[1]),
+                                  int(rope_split[2]), float(rope_theta), float(eps), _dtype_code(q_raw), int(block),
+                                  qbar_out.data_ptr(), kbar_out.data_ptr(), _stream_handle(stream))
+    _check(st, "sol_qk_prologue_pool")
+    return q_out, k_out, qbar_out, kbar_out
+
+
+def sol_block_select_pooled(qbar, kbar, grid, block, topk, idx_out=None, return_scores=False, stream=None):
+    """Scores + top-k from block means [B, H, nb, D] (fp32).  Returns idx (and the scores)."""
+    _cuda(qbar, "qbar"), _cuda(kbar, "kbar")
+    if qbar.dtype != torch.float32 or kbar.dtype != torch.float32:
+        raise TypeError("qbar and kbar must be float32")
+    B, H, nb, D = qbar.shape
+    N = int(grid[0]) * int(grid[1]) * int(grid[2])
+    s = SolShape(B, N, H, D, int(grid[0]), int(grid[1]), int(grid[2]))
+    if idx_out is None:
+        idx_out = torch.empty((B, H, nb, topk), dtype=torch.int32, device=qbar.device)
+    scores = torch.empty((B, H, nb, nb), dtype=torch.float32, device=qbar.device) if return_scores else None
+    st = lib.sol_block_select_pooled(qbar.data_ptr(), kbar.data_ptr(), s, int(block), int(topk),
+                                     _cuda(idx_out, "idx_out").data_ptr(),
+                                     scores.data_ptr() if scores is not None else None, _stream_handle(stream))
+    _check(st, "sol_block_select_pooled")
+    return (idx_out, scores) if return_scores else idx_out
 
 
 def sol_block_select_workspace_bytes(shape: SolShape, block: int) -> int:

@@ -181,5 +181,132 @@ __global__ void __launch_bounds__(256, sizeof(T) == 2 ? 3 : 4) qk_prologue_kerne
   }
 }
 
+// ------------------------------------------------------------------ prologue + block pooling
+// The same prologue, organised by key block so that the pooled means of the
+// selection come out of the same pass over Q and K: one CTA per (b, block i)
+// takes the block's tokens for every head.  Row group g works on heads g, g +
+// GPC, ... (consecutive groups on consecutive heads, so a warp moves 512
+// contiguous bytes per token); for each head it writes the block's output rows
+// and then the fp32 mean over the block's valid tokens of the stored (rounded)
+// outputs, which is what the selection pools.
+__device__ __forceinline__ void store_vec_acc(float* p, const float (&y)[4], float (&acc)[4]) {
+  store_vec(p, y);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) acc[e] += y[e];
+}
+__device__ __forceinline__ void store_vec_acc(__nv_bfloat16* p, const float (&y)[8], float (&acc)[8]) {
+  uint32_t w[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    w[e] = bf16x2_bits(y[2 * e], y[2 * e + 1]);
+    acc[2 * e] += __uint_as_float(w[e] << 16);             // the stored (rounded) values
+    acc[2 * e + 1] += __uint_as_float(w[e] & 0xFFFF0000u);
+  }
+  *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// grid (nb, B); qbar, kbar: fp32 [B, H, nb, D].
+template <typename T, int D>
+__global__ void __launch_bounds__(256) qk_prologue_pool_kernel(const Params p, int block, int nb, float* qbar,
+                                                               float* kbar) {
+  extern __shared__ float2 tab[];   // [gt * dt/2 | gh * dh/2 | gw * dw/2] of (cos, sin)
+  const int pt = p.dt / 2, ph = p.dh / 2, pw = p.dw / 2;
+  for (int i = threadIdx.x; i < p.tab_total; i += blockDim.x) {
+    int pos, pair, d_axis;
+    if (i < p.tab_t) { pos = i / pt; pair = i % pt; d_axis = p.dt; }
+    else if (i < p.tab_h) { pos = (i - p.tab_t) / ph; pair = (i - p.tab_t) % ph; d_axis = p.dh; }
+    else { pos = (i - p.tab_h) / pw; pair = (i - p.tab_h) % pw; d_axis = p.dw; }
+    const double angle = static_cast<double>(pos) * exp2(-p.log2_theta * (2.0 * pair) / d_axis);
+    double s, c;
+    sincos(angle, &s, &c);
+    tab[i] = make_float2(static_cast<float>(c), static_cast<float>(s));
+  }
+  __syncthreads();
+
+  constexpr int V = Vec<T>::n;
+  constexpr int L = D / V;            // lanes per row
+  constexpr int GPC = 256 / L;        // row groups per CTA
+  const int lane_in_row = threadIdx.x % L;
+  const unsigned lane = threadIdx.x & 31u;
+  const unsigned seg = (L == 32) ? 0xffffffffu : (((1u << (L & 31)) - 1u) << (lane & ~(unsigned)(L - 1)));
+  const int grp = threadIdx.x / L;
+  const int bi = blockIdx.x, b = blockIdx.y;
+  const int n0 = bi * block;
+  const int n1 = min(n0 + block, p.N);
+  const float inv = 1.0f / static_cast<float>(n1 - n0);
+
+  int axis[V / 2], slot[V / 2];
+#pragma unroll
+  for (int e = 0; e < V / 2; ++e) {
+    const int c = lane_in_row * V + 2 * e;
+    if (c < p.dt) { axis[e] = 0; slot[e] = c / 2; }
+    else if (c < p.dt + p.dh) { axis[e] = 1; slot[e] = p.tab_t + (c - p.dt) / 2; }
+    else { axis[e] = 2; slot[e] = p.tab_h + (c - p.dt - p.dh) / 2; }
+  }
+  const T* qi = static_cast<const T*>(p.q_in);
+  const T* ki = static_cast<const T*>(p.k_in);
+  T* qo = static_cast<T*>(p.q_out);
+  T* ko = static_cast<T*>(p.k_out);
+  const int hw = p.gh * p.gw;
+  auto angles = [&](int n, float2 (&cs)[V / 2]) {
+    const int t = n / hw, y = (n / p.gw) % p.gh, x = n % p.gw;
+    const int st = t * pt, sy = y * ph, sx = x * pw;
+#pragma unroll
+    for (int e = 0; e < V / 2; ++e) cs[e] = tab[slot[e] + (axis[e] == 0 ? st : (axis[e] == 1 ? sy : sx))];
+  };
+
+  for (int h = grp; h < p.H; h += GPC) {
+    float gq[V], gk[V], aq[V], ak[V];
+#pragma unroll
+    for (int e = 0; e < V; ++e) {
+      gq[e] = __ldg(p.gamma_q + h * D + lane_in_row * V + e);
+      gk[e] = __ldg(p.gamma_k + h * D + lane_in_row * V + e);
+      aq[e] = 0.f;
+      ak[e] = 0.f;
+    }
+    const size_t base = (static_cast<size_t>(b) * p.N * p.H + h) * D + lane_in_row * V;
+    const size_t tstride = static_cast<size_t>(p.H) * D;
+    int n = n0;
+    for (; n + 1 < n1; n += 2) {   // two tokens in flight
+      const size_t o1 = base + static_cast<size_t>(n) * tstride, o2 = o1 + tstride;
+      float xq1[V], xk1[V], xq2[V], xk2[V];
+      load_vec(qi + o1, xq1);
+      load_vec(ki + o1, xk1);
+      load_vec(qi + o2, xq2);
+      load_vec(ki + o2, xk2);
+      float2 cs1[V / 2], cs2[V / 2];
+      angles(n, cs1);
+      angles(n + 1, cs2);
+      norm_rotate<V, L>(xq1, gq, cs1, seg, D, p.eps);
+      norm_rotate<V, L>(xk1, gk, cs1, seg, D, p.eps);
+      norm_rotate<V, L>(xq2, gq, cs2, seg, D, p.eps);
+      norm_rotate<V, L>(xk2, gk, cs2, seg, D, p.eps);
+      store_vec_acc(qo + o1, xq1, aq);
+      store_vec_acc(ko + o1, xk1, ak);
+      store_vec_acc(qo + o2, xq2, aq);
+      store_vec_acc(ko + o2, xk2, ak);
+    }
+    if (n < n1) {
+      const size_t o1 = base + static_cast<size_t>(n) * tstride;
+      float xq[V], xk[V];
+      load_vec(qi + o1, xq);
+      load_vec(ki + o1, xk);
+      float2 cs[V / 2];
+      angles(n, cs);
+      norm_rotate<V, L>(xq, gq, cs, seg, D, p.eps);
+      norm_rotate<V, L>(xk, gk, cs, seg, D, p.eps);
+      store_vec_acc(qo + o1, xq, aq);
+      store_vec_acc(ko + o1, xk, ak);
+    }
+    float* dq = qbar + ((static_cast<size_t>(b) * p.H + h) * nb + bi) * D + lane_in_row * V;
+    float* dk = kbar + ((static_cast<size_t>(b) * p.H + h) * nb + bi) * D + lane_in_row * V;
+#pragma unroll
+    for (int e = 0; e < V; e += 4) {
+      *reinterpret_cast<float4*>(dq + e) = make_float4(aq[e] * inv, aq[e + 1] * inv, aq[e + 2] * inv, aq[e + 3] * inv);
+      *reinterpret_cast<float4*>(dk + e) = make_float4(ak[e] * inv, ak[e + 1] * inv, ak[e + 2] * inv, ak[e + 3] * inv);
+    }
+  }
+}
+
 }  // namespace prologue
 }  // namespace sol

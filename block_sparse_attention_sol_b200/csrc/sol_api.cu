@@ -111,6 +111,26 @@ __global__ void wait_timeout_selftest_kernel(unsigned long long limit_ns) {
 
 namespace {
 
+// Launch shape of the score / top-k kernel: 32 rows per CTA when their scores
+// fit in shared memory, else 16; keys per lane for the top-k.
+struct ScorePlan {
+  int rpw = 4, kpl = 8;
+  size_t smem = 0;
+  dim3 grid;
+};
+
+sol_status plan_scores(const sol_shape& s, int nb, ScorePlan* plan) {
+  if (s.D != 64 && s.D != 128) return SOL_ERR_UNSUPPORTED;
+  if (nb > sol::select::kMaxNb) return SOL_ERR_UNSUPPORTED;
+  if (static_cast<long long>(s.B) * s.H > 65535) return SOL_ERR_UNSUPPORTED;
+  plan->rpw = sol::select::score_topk_smem_bytes(s.D, 32, nb) <= kMaxSmemPerBlock ? 4 : 2;
+  plan->smem = sol::select::score_topk_smem_bytes(s.D, 8 * plan->rpw, nb);
+  if (plan->smem > kMaxSmemPerBlock) return SOL_ERR_UNSUPPORTED;
+  plan->kpl = nb <= 256 ? 8 : nb <= 512 ? 16 : nb <= 1024 ? 32 : 64;
+  plan->grid = dim3((nb + 8 * plan->rpw - 1) / (8 * plan->rpw), s.B * s.H);
+  return SOL_OK;
+}
+
 // Launches score_topk_kernel<D, RPW, KPL> for the runtime choices (shared-memory
 // opt-in set once per device and instantiation).
 template <int D, int RPW, int KPL>
@@ -150,6 +170,41 @@ sol_status launch_score_topk(DeviceInfo* di, int D, int rpw, int kpl, dim3 grid,
 
 }  // namespace
 
+namespace {
+
+// Argument checks and kernel parameters shared by both prologue entry points.
+sol_status prologue_params(const void* q_raw, const void* k_raw, void* q_out, void* k_out, const float* gamma_q,
+                           const float* gamma_k, sol_shape s, int rope_dt, int rope_dh, int rope_dw, float rope_theta,
+                           float eps, sol_dtype dt, sol::prologue::Params* out, size_t* smem_out) {
+  if (!q_raw || !k_raw || !q_out || !k_out || !gamma_q || !gamma_k) return SOL_ERR_INVALID_ARG;
+  if (!aligned16(q_raw) || !aligned16(k_raw) || !aligned16(q_out) || !aligned16(k_out)) return SOL_ERR_INVALID_ARG;
+  if (!shape_ok(s)) return SOL_ERR_INVALID_ARG;
+  if (dt != SOL_F32 && dt != SOL_BF16) return SOL_ERR_INVALID_ARG;
+  if (rope_dt < 0 || rope_dh < 0 || rope_dw < 0 || (rope_dt | rope_dh | rope_dw) & 1) return SOL_ERR_INVALID_ARG;
+  if (rope_dt + rope_dh + rope_dw != s.D) return SOL_ERR_INVALID_ARG;
+  if (!(rope_theta > 0.f) || !(eps >= 0.f) || !std::isfinite(rope_theta) || !std::isfinite(eps))
+    return SOL_ERR_INVALID_ARG;
+  if (s.D != 64 && s.D != 128) return SOL_ERR_UNSUPPORTED;
+  if (static_cast<long long>(s.B) * s.N >= (1ll << 31)) return SOL_ERR_UNSUPPORTED;
+  sol::prologue::Params& p = *out;
+  p.q_in = q_raw; p.k_in = k_raw; p.q_out = q_out; p.k_out = k_out;
+  p.gamma_q = gamma_q; p.gamma_k = gamma_k;
+  p.tokens = s.B * s.N;
+  p.N = s.N; p.H = s.H;
+  p.gt = s.grid_t; p.gh = s.grid_h; p.gw = s.grid_w;
+  p.dt = rope_dt; p.dh = rope_dh; p.dw = rope_dw;
+  p.log2_theta = std::log2(static_cast<double>(rope_theta));
+  p.eps = eps;
+  p.tab_t = s.grid_t * (rope_dt / 2);
+  p.tab_h = p.tab_t + s.grid_h * (rope_dh / 2);
+  p.tab_total = p.tab_h + s.grid_w * (rope_dw / 2);
+  *smem_out = static_cast<size_t>(p.tab_total) * sizeof(float2);
+  if (*smem_out > 48 * 1024) return SOL_ERR_UNSUPPORTED;
+  return SOL_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 const char* sol_status_string(sol_status st) {
@@ -166,32 +221,11 @@ const char* sol_status_string(sol_status st) {
 sol_status sol_qk_prologue(const void* q_raw, const void* k_raw, void* q_out, void* k_out, const float* gamma_q,
                            const float* gamma_k, sol_shape s, int rope_dt, int rope_dh, int rope_dw, float rope_theta,
                            float eps, sol_dtype dt, cudaStream_t stream) {
-  if (!q_raw || !k_raw || !q_out || !k_out || !gamma_q || !gamma_k) return SOL_ERR_INVALID_ARG;
-  if (!aligned16(q_raw) || !aligned16(k_raw) || !aligned16(q_out) || !aligned16(k_out)) return SOL_ERR_INVALID_ARG;
-  if (!shape_ok(s)) return SOL_ERR_INVALID_ARG;
-  if (dt != SOL_F32 && dt != SOL_BF16) return SOL_ERR_INVALID_ARG;
-  if (rope_dt < 0 || rope_dh < 0 || rope_dw < 0 || (rope_dt | rope_dh | rope_dw) & 1) return SOL_ERR_INVALID_ARG;
-  if (rope_dt + rope_dh + rope_dw != s.D) return SOL_ERR_INVALID_ARG;
-  if (!(rope_theta > 0.f) || !(eps >= 0.f) || !std::isfinite(rope_theta) || !std::isfinite(eps))
-    return SOL_ERR_INVALID_ARG;
-  if (s.D != 64 && s.D != 128) return SOL_ERR_UNSUPPORTED;
-
-  if (static_cast<long long>(s.B) * s.N >= (1ll << 31)) return SOL_ERR_UNSUPPORTED;
   sol::prologue::Params p;
-  p.q_in = q_raw; p.k_in = k_raw; p.q_out = q_out; p.k_out = k_out;
-  p.gamma_q = gamma_q; p.gamma_k = gamma_k;
-  p.tokens = s.B * s.N;
-  p.N = s.N; p.H = s.H;
-  p.gt = s.grid_t; p.gh = s.grid_h; p.gw = s.grid_w;
-  p.dt = rope_dt; p.dh = rope_dh; p.dw = rope_dw;
-  p.log2_theta = std::log2(static_cast<double>(rope_theta));
-  p.eps = eps;
-  p.tab_t = s.grid_t * (rope_dt / 2);
-  p.tab_h = p.tab_t + s.grid_h * (rope_dh / 2);
-  p.tab_total = p.tab_h + s.grid_w * (rope_dw / 2);
-  const size_t smem = static_cast<size_t>(p.tab_total) * sizeof(float2);
-  if (smem > 48 * 1024) return SOL_ERR_UNSUPPORTED;
-
+  size_t smem = 0;
+  if (sol_status st = prologue_params(q_raw, k_raw, q_out, k_out, gamma_q, gamma_k, s, rope_dt, rope_dh, rope_dw,
+                                      rope_theta, eps, dt, &p, &smem))
+    return st;
   DeviceInfo* di = nullptr;
   if (sol_status st = device_info(&di)) return st;
   // Every row group keeps one head: the number of groups must be a multiple of H.
@@ -217,6 +251,35 @@ sol_status sol_qk_prologue(const void* q_raw, const void* k_raw, void* q_out, vo
   return launch_status();
 }
 
+sol_status sol_qk_prologue_pool(const void* q_raw, const void* k_raw, void* q_out, void* k_out, const float* gamma_q,
+                                const float* gamma_k, sol_shape s, int rope_dt, int rope_dh, int rope_dw,
+                                float rope_theta, float eps, sol_dtype dt, int block, float* qbar_out,
+                                float* kbar_out, cudaStream_t stream) {
+  sol::prologue::Params p;
+  size_t smem = 0;
+  if (sol_status st = prologue_params(q_raw, k_raw, q_out, k_out, gamma_q, gamma_k, s, rope_dt, rope_dh, rope_dw,
+                                      rope_theta, eps, dt, &p, &smem))
+    return st;
+  if (!qbar_out || !kbar_out || !aligned16(qbar_out) || !aligned16(kbar_out) || block <= 0)
+    return SOL_ERR_INVALID_ARG;
+  const int nb = num_blocks(s.N, block);
+  if (nb > 65535 || s.B > 65535) return SOL_ERR_UNSUPPORTED;
+  const dim3 grid(nb, s.B);
+  if (dt == SOL_BF16) {
+    if (s.D == 128)
+      sol::prologue::qk_prologue_pool_kernel<__nv_bfloat16, 128><<<grid, 256, smem, stream>>>(p, block, nb, qbar_out,
+                                                                                              kbar_out);
+    else
+      sol::prologue::qk_prologue_pool_kernel<__nv_bfloat16, 64><<<grid, 256, smem, stream>>>(p, block, nb, qbar_out,
+                                                                                             kbar_out);
+  } else {
+    if (s.D == 128)
+      sol::prologue::qk_prologue_pool_kernel<float, 128><<<grid, 256, smem, stream>>>(p, block, nb, qbar_out, kbar_out);
+    else
+      sol::prologue::qk_prologue_pool_kernel<float, 64><<<grid, 256, smem, stream>>>(p, block, nb, qbar_out, kbar_out);
+  }
+  return launch_status();
+}
 
 size_t sol_block_select_workspace_bytes(sol_shape s, int block) {
   if (!shape_ok(s) || block <= 0) return 0;
@@ -234,9 +297,8 @@ sol_status sol_block_select(const void* q, const void* k, sol_shape s, int block
   const int nb = num_blocks(s.N, block);
   if (topk < 1 || topk > nb) return SOL_ERR_INVALID_ARG;
   if (workspace_bytes < sol_block_select_workspace_bytes(s, block)) return SOL_ERR_INVALID_ARG;
-  if (s.D != 64 && s.D != 128) return SOL_ERR_UNSUPPORTED;
-  if (nb > 2048) return SOL_ERR_UNSUPPORTED;
-  if (static_cast<long long>(s.B) * s.H > 65535) return SOL_ERR_UNSUPPORTED;
+  ScorePlan plan;
+  if (sol_status st = plan_scores(s, nb, &plan)) return st;
 
   DeviceInfo* di = nullptr;
   if (sol_status st = device_info(&di)) return st;
@@ -252,14 +314,24 @@ sol_status sol_block_select(const void* q, const void* k, sol_shape s, int block
                                                                   static_cast<const float*>(k), qbar, kbar, s.N, s.H,
                                                                   s.D, block, nb);
   if (sol_status st = launch_status()) return st;
+  return launch_score_topk(di, s.D, plan.rpw, plan.kpl, plan.grid, plan.smem, stream, qbar, kbar, idx_out,
+                           scores_out, nb, topk);
+}
 
-  // 32 rows per CTA when their scores fit in shared memory, else 16.
-  const int rpw = sol::select::score_topk_smem_bytes(s.D, 32, nb) <= kMaxSmemPerBlock ? 4 : 2;
-  const size_t smem = sol::select::score_topk_smem_bytes(s.D, 8 * rpw, nb);
-  if (smem > kMaxSmemPerBlock) return SOL_ERR_UNSUPPORTED;
-  const int kpl = nb <= 256 ? 8 : nb <= 512 ? 16 : nb <= 1024 ? 32 : 64;
-  const dim3 sg((nb + 8 * rpw - 1) / (8 * rpw), s.B * s.H);
-  return launch_score_topk(di, s.D, rpw, kpl, sg, smem, stream, qbar, kbar, idx_out, scores_out, nb, topk);
+sol_status sol_block_select_pooled(const float* qbar, const float* kbar, sol_shape s, int block, int topk,
+                                   int32_t* idx_out, float* scores_out, cudaStream_t stream) {
+  if (!qbar || !kbar || !idx_out) return SOL_ERR_INVALID_ARG;
+  if (!aligned16(qbar) || !aligned16(kbar) || !aligned16(idx_out)) return SOL_ERR_INVALID_ARG;
+  if (scores_out && !aligned16(scores_out)) return SOL_ERR_INVALID_ARG;
+  if (!shape_ok(s) || block <= 0) return SOL_ERR_INVALID_ARG;
+  const int nb = num_blocks(s.N, block);
+  if (topk < 1 || topk > nb) return SOL_ERR_INVALID_ARG;
+  ScorePlan plan;
+  if (sol_status st = plan_scores(s, nb, &plan)) return st;
+  DeviceInfo* di = nullptr;
+  if (sol_status st = device_info(&di)) return st;
+  return launch_score_topk(di, s.D, plan.rpw, plan.kpl, plan.grid, plan.smem, stream, qbar, kbar, idx_out,
+                           scores_out, nb, topk);
 }
 
 sol_status sol_sparse_attn_fwd(const void* q, const void* k, const void* v, const int32_t* idx, sol_shape s,

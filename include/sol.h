@@ -101,6 +101,38 @@ sol_status sol_block_select(const void* q, const void* k, sol_shape s, int block
                             void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * sol_qk_prologue_pool -- sol_qk_prologue that also emits the block means the
+ * selection pools, from the same pass over Q and K (the runtime on the pages
+ * made this "preparation" 76.4% faster: ai-feiten.nl, same section).
+ *
+ * q_out, k_out : exactly sol_qk_prologue's outputs (same arithmetic, bit for bit).
+ * qbar_out[b,h,i,:] = mean over the valid tokens n of block i of the STORED
+ *                     (rounded) q_out[b,n,h,:], fp32 [B, H, nb, D], nb =
+ *                     ceil(N/block); kbar_out likewise from k_out.  Summed in
+ *                     ascending token order in fp32, so they equal the means
+ *                     sol_block_select computes from q_out and k_out.
+ * Other arguments, aliasing and limits as for sol_qk_prologue; block >= 1;
+ * qbar_out, kbar_out 16-byte aligned, caller-owned.
+ */
+sol_status sol_qk_prologue_pool(const void* q_raw, const void* k_raw, void* q_out, void* k_out,
+                                const float* gamma_q, const float* gamma_k, sol_shape s,
+                                int rope_dt, int rope_dh, int rope_dw, float rope_theta, float eps,
+                                sol_dtype dt, int block, float* qbar_out, float* kbar_out,
+                                cudaStream_t stream);
+
+/*
+ * sol_block_select_pooled -- the scoring and top-k of sol_block_select from
+ * block means already computed (by sol_qk_prologue_pool): no pooling pass and
+ * no workspace.
+ *
+ * qbar, kbar : fp32 [B, H, nb, D], 16-byte aligned.  idx_out, scores_out and
+ * the limits as for sol_block_select.  Given equal means, the result equals
+ * sol_block_select's.
+ */
+sol_status sol_block_select_pooled(const float* qbar, const float* kbar, sol_shape s, int block, int topk,
+                                   int32_t* idx_out, float* scores_out, cudaStream_t stream);
+
+/*
  * sol_sparse_attn_fwd -- Sol-Attn block-sparse attention forward
  * (ai-feiten.nl, same section: attention restricted, per query, to the parts
  * that matter).

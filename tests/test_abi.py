@@ -114,3 +114,37 @@ def test_status_strings(lib):
     f.argtypes = [ctypes.c_int]
     assert [f(i).decode() for i in range(5)] == ["SOL_OK", "SOL_ERR_INVALID_ARG", "SOL_ERR_UNSUPPORTED",
                                                  "SOL_ERR_CUDA", "SOL_ERR_TIMEOUT"]
+
+
+def test_prologue_pool_argument_checks(lib):
+    f = lib.sol_qk_prologue_pool
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p] * 6 + [Shape, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float,
+                                          ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
+                                          ctypes.c_void_p, ctypes.c_void_p]
+
+    def call(ptr=FAKE, shape=OK_SHAPE, split=(24, 20, 20), block=64, qbar=FAKE, kbar=FAKE):
+        return f(ptr, FAKE, FAKE, FAKE, FAKE, FAKE, shape, *split, 10000.0, 1e-6, 0, block, qbar, kbar, None)
+
+    assert call(ptr=None) == INVALID                       # the prologue's own checks apply
+    assert call(split=(24, 20, 18)) == INVALID
+    assert call(block=0) == INVALID
+    assert call(qbar=None) == INVALID
+    assert call(kbar=MISALIGNED) == INVALID
+    assert call(shape=Shape(1, 1024, 2, 96, 4, 16, 16), split=(32, 32, 32)) == UNSUPPORTED
+
+
+def test_select_pooled_argument_checks(lib):
+    f = lib.sol_block_select_pooled
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p, ctypes.c_void_p, Shape, ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
+                  ctypes.c_void_p, ctypes.c_void_p]
+    assert f(FAKE, FAKE, OK_SHAPE, 64, 0, FAKE, None, None) == INVALID          # k = 0
+    assert f(FAKE, FAKE, OK_SHAPE, 64, 17, FAKE, None, None) == INVALID         # k > nb
+    assert f(None, FAKE, OK_SHAPE, 64, 4, FAKE, None, None) == INVALID
+    assert f(FAKE, MISALIGNED, OK_SHAPE, 64, 4, FAKE, None, None) == INVALID
+    assert f(FAKE, FAKE, OK_SHAPE, 64, 4, None, None, None) == INVALID          # no idx_out
+    assert f(FAKE, FAKE, OK_SHAPE, 64, 4, FAKE, MISALIGNED, None) == INVALID    # misaligned scores_out
+    assert f(FAKE, FAKE, Shape(1, 1000, 2, 64, 4, 16, 16), 64, 4, FAKE, None, None) == INVALID
+    big = Shape(1, 2049 * 64, 2, 64, 1, 2049, 64)                                 # nb = 2049 > 2048
+    assert f(FAKE, FAKE, big, 64, 4, FAKE, None, None) == UNSUPPORTED

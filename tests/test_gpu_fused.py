@@ -1,0 +1,81 @@
+"""GPU parity of the fused preparation path: sol_qk_prologue_pool followed by
+sol_block_select_pooled.
+
+  * Its Q / K outputs are those of sol_qk_prologue, bit for bit.
+  * Its block means are the oracle's block means of those stored outputs, within
+    the error bound of an fp32 running sum of <= block values followed by one
+    multiplication by the rounded reciprocal of the count:
+        |r - m| <= gamma_(n-1) * mean|x| * (1 + 3u) + 3u |m|,  u = 2^-24,
+    gamma_k = k u / (1 - k u)  (recursive summation bound).
+  * Its selection equals sol_block_select's on the same prologue outputs, id for
+    id (both pool in ascending token order in fp32), and so passes the same
+    oracle selection rule.
+Covered: the fp32 workload (4x16x16 grid, block 64, k = 4 and 16), a small bf16
+case with a ragged last block, and the 896x512 workload at full size.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as orc
+from tests.gpu_common import check_selection, cpu_inputs, np64
+from workloads import WORKLOADS, make_inputs, Workload
+
+pytestmark = pytest.mark.gpu
+
+U32 = 2.0 ** -24
+
+
+def pooled_tolerance(x64: np.ndarray, block: int) -> tuple[np.ndarray, np.ndarray]:
+    """Oracle block means of x [B, N, H, D] and the fp32 kernel's error bound."""
+    m = orc.block_pool(x64, block)
+    mean_abs = orc.block_pool(np.abs(x64), block)
+    k = block - 1
+    gamma = k * U32 / (1 - k * U32)
+    return m, gamma * mean_abs * (1 + 3 * U32) + 3 * U32 * np.abs(m)
+
+
+def run_case(sol, wl: Workload, inp, topks):
+    q_raw, k_raw = inp["q"].cuda(), inp["k"].cuda()
+    gq, gk = inp["gamma_q"].cuda(), inp["gamma_k"].cuda()
+    args = (wl.grid,)
+    q_ref, k_ref = sol.sol_qk_prologue(q_raw, k_raw, gq, gk, *args, wl.rope_split, wl.rope_theta, wl.eps)
+    q, k, qbar, kbar = sol.sol_qk_prologue_pool(q_raw, k_raw, gq, gk, wl.grid, wl.block, wl.rope_split,
+                                                wl.rope_theta, wl.eps)
+    torch.cuda.synchronize()
+    assert torch.equal(q.view(torch.int16) if q.dtype == torch.bfloat16 else q,
+                       q_ref.view(torch.int16) if q_ref.dtype == torch.bfloat16 else q_ref)
+    assert torch.equal(k.view(torch.int16) if k.dtype == torch.bfloat16 else k,
+                       k_ref.view(torch.int16) if k_ref.dtype == torch.bfloat16 else k_ref)
+    assert qbar.shape == (wl.B, wl.H, wl.nb, wl.D)
+    for out, bar in ((q, qbar), (k, kbar)):
+        m, tol = pooled_tolerance(np64(out), wl.block)
+        err = np.abs(np64(bar) - m)
+        assert (err <= tol).all(), float((err - tol).max())
+    for topk in topks:
+        idx_f, s_f = sol.sol_block_select_pooled(qbar, kbar, wl.grid, wl.block, topk, return_scores=True)
+        idx_u, s_u = sol.sol_block_select(q, k, wl.grid, wl.block, topk, return_scores=True)
+        torch.cuda.synchronize()
+        assert torch.equal(s_f, s_u)
+        assert torch.equal(idx_f, idx_u)
+        if wl.config_id == 0:   # and the oracle's selection rule on the stored outputs
+            _, s_ref = orc.block_select(np64(q), np64(k), wl.block, topk)
+            check_selection(idx_f.cpu().numpy(), s_ref, topk)
+
+
+def test_fused_workload0_fp32(sol):
+    wl = WORKLOADS[0]
+    run_case(sol, wl, cpu_inputs(0), wl.topk)
+
+
+def test_fused_small_bf16_ragged_block(sol):
+    # 3 x 8 x 40 grid = 960 tokens: 7 full blocks of 128 and a last block of 64
+    wl = Workload(config_id=90, name="small bf16, ragged last block", dtype="bf16", B=2, H=4, D=128,
+                  grid=(3, 8, 40), block=128, topk=(3,))
+    assert wl.N % wl.block == 64
+    run_case(sol, wl, make_inputs(wl, seed=5), (1, 3, wl.nb))
+
+
+def test_fused_workload1_bf16_full(sol):
+    wl = WORKLOADS[1]
+    run_case(sol, wl, cpu_inputs(1), wl.topk)
