@@ -152,15 +152,30 @@ __global__ void __launch_bounds__(kThreads, 1) score_topk_kernel(const float* __
   }
   const int lane = threadIdx.x & 31;
   const int rg = (threadIdx.x >> 5) * RPW;   // this warp's rows
+  // Key chunks are double-buffered through registers: the next chunk's global
+  // loads are in flight while the current chunk's FMAs run.
+  constexpr int kPre = kKeys * (D / 4) / kThreads;   // float4 per thread per chunk
+  float4 pre[kPre];
+  auto load_chunk = [&](int j0) {
+#pragma unroll
+    for (int u = 0; u < kPre; ++u) {
+      const int e = threadIdx.x + u * kThreads;
+      const int j = e / (D / 4), d = (e % (D / 4)) * 4;
+      pre[u] = j0 + j < nb ? __ldg(reinterpret_cast<const float4*>(kb + static_cast<size_t>(j0 + j) * D + d))
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  };
+  load_chunk(0);
   for (int j0 = 0; j0 < nb; j0 += kKeys) {
     __syncthreads();   // previous chunk fully consumed (and qs written, the first time)
-    for (int e = threadIdx.x; e < kKeys * (D / 4); e += kThreads) {
+#pragma unroll
+    for (int u = 0; u < kPre; ++u) {
+      const int e = threadIdx.x + u * kThreads;
       const int j = e / (D / 4), d = (e % (D / 4)) * 4;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (j0 + j < nb) v = __ldg(reinterpret_cast<const float4*>(kb + static_cast<size_t>(j0 + j) * D + d));
-      *reinterpret_cast<float4*>(ks + j * P + d) = v;
+      *reinterpret_cast<float4*>(ks + j * P + d) = pre[u];
     }
     __syncthreads();
+    if (j0 + kKeys < nb) load_chunk(j0 + kKeys);
     float acc[RPW][4];   // [row][key lane + 32 c]
 #pragma unroll
     for (int r = 0; r < RPW; ++r)

@@ -79,3 +79,33 @@ def test_fused_small_bf16_ragged_block(sol):
 def test_fused_workload1_bf16_full(sol):
     wl = WORKLOADS[1]
     run_case(sol, wl, cpu_inputs(1), wl.topk)
+
+
+def test_host_pipeline_matches_direct_calls(sol):
+    """Clips streamed through HostChainPipeline (three streams, double-buffered
+    device buffers) give exactly the outputs of the direct fused chain on each clip."""
+    from block_sparse_attention_sol_b200.pipeline import HostChainPipeline
+    wl = Workload(config_id=91, name="pipeline check, ragged last block", dtype="bf16", B=1, H=4, D=128,
+                  grid=(3, 8, 40), block=128, topk=(3,))
+    topk = 3
+    clips = [make_inputs(wl, seed=s) for s in range(5)]
+    gq, gk = clips[0]["gamma_q"].cuda(), clips[0]["gamma_k"].cuda()
+    pipe = HostChainPipeline(wl.B, wl.N, wl.H, wl.D, wl.grid, wl.block, topk, gq, gk, rope_split=wl.rope_split,
+                             rope_theta=wl.rope_theta, eps=wl.eps)
+    outs = []
+    for c in clips:
+        host = {n: c[n].pin_memory() for n in ("q", "k", "v")}
+        o_host = torch.empty(c["q"].shape, dtype=c["q"].dtype).pin_memory()
+        lse_host = torch.empty((wl.B, wl.H, wl.N), dtype=torch.float32).pin_memory()
+        pipe.submit(host["q"], host["k"], host["v"], o_host, lse_host)
+        outs.append((host, o_host, lse_host))
+    pipe.synchronize()
+    for c, (_, o_host, lse_host) in zip(clips, outs):
+        q, k, qbar, kbar = sol.sol_qk_prologue_pool(c["q"].cuda(), c["k"].cuda(), gq, gk, wl.grid, wl.block,
+                                                    wl.rope_split, wl.rope_theta, wl.eps)
+        idx = sol.sol_block_select_pooled(qbar, kbar, wl.grid, wl.block, topk)
+        o, lse = sol.sol_sparse_attn_fwd(q, k, c["v"].cuda(), idx, wl.grid, wl.block)
+        torch.cuda.synchronize()
+        assert torch.equal(o.cpu().view(torch.int16), o_host.view(torch.int16))
+        assert torch.equal(lse.cpu(), lse_host)
+    assert sol.sol_check_device_status() == sol.SOL_OK
