@@ -11,10 +11,10 @@
 //           each thread computes 4 rows x 4 keys of a 128-key chunk: 16-byte
 //           shared loads, rows broadcast across the warp, keys 32 apart.
 //   top-k:  per row, the k largest scores, exact ties to the lower j, written in
-//           ascending j.  A warp holds the row's order-preserving keys in
-//           registers, finds the k-th largest by a most-significant-bit-first
-//           search of the 32-bit key space, then compacts the winners in
-//           ascending j with ballots.
+//           ascending j.  A warp holds two rows' order-preserving keys in
+//           registers, finds each row's k-th largest by a most-significant-bit-
+//           first search of the 32-bit key space (the two searches interleaved),
+//           then compacts the winners in ascending j with ballots.
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -91,20 +91,39 @@ __device__ __forceinline__ uint32_t order_key(float f) {
 // The k-th largest key of a row held as KPL keys per lane (key j at lane j % 32,
 // slot j / 32; 0 pads, below every real key), then the row's ids with key above
 // it, plus the first (topk - count above) with key equal to it, in ascending j.
-template <int KPL>
-__device__ __forceinline__ void topk_row(const uint32_t (&key)[KPL], int nb, int topk, int32_t* out, int lane) {
-  uint32_t prefix = 0u;   // largest T with count(key >= T) >= topk, built bit by bit
+// The k-th largest key of each of NR rows held as KPL keys per lane (key j at
+// lane j % 32, slot j / 32; 0 pads, below every real key): the largest T with
+// count(key >= T) >= topk, built most significant bit first.  The NR searches
+// share one bit loop so that their counts and warp reductions overlap.
+template <int KPL, int NR>
+__device__ __forceinline__ void kth_largest(const uint32_t (&key)[NR][KPL], int topk, uint32_t (&prefix)[NR]) {
+#pragma unroll
+  for (int r = 0; r < NR; ++r) prefix[r] = 0u;
 #pragma unroll 1
   for (int bit = 31; bit >= 0; --bit) {
-    const uint32_t cand = prefix | (1u << bit);
-    uint32_t cnt = 0;
+    uint32_t cnt[NR];
 #pragma unroll
-    for (int q = 0; q < KPL; ++q) cnt += key[q] >= cand ? 1u : 0u;
-    if (static_cast<int>(__reduce_add_sync(0xffffffffu, cnt)) >= topk) prefix = cand;
+    for (int r = 0; r < NR; ++r) {
+      const uint32_t cand = prefix[r] | (1u << bit);
+      uint32_t c = 0;
+#pragma unroll
+      for (int q = 0; q < KPL; ++q) c += key[r][q] >= cand ? 1u : 0u;
+      cnt[r] = c;
+    }
+#pragma unroll
+    for (int r = 0; r < NR; ++r)
+      if (static_cast<int>(__reduce_add_sync(0xffffffffu, cnt[r])) >= topk) prefix[r] |= 1u << bit;
   }
+}
+
+// The row's ids with key above `kth`, plus the first (topk - count above) with
+// key equal to it, written in ascending j.
+template <int KPL>
+__device__ __forceinline__ void compact_row(const uint32_t (&key)[KPL], uint32_t kth, int nb, int topk, int32_t* out,
+                                            int lane) {
   uint32_t gt = 0;
 #pragma unroll
-  for (int q = 0; q < KPL; ++q) gt += key[q] > prefix ? 1u : 0u;
+  for (int q = 0; q < KPL; ++q) gt += key[q] > kth ? 1u : 0u;
   const int need_eq = topk - static_cast<int>(__reduce_add_sync(0xffffffffu, gt));
   const uint32_t lt_mask = (1u << lane) - 1u;
   int written = 0, eq_seen = 0;
@@ -112,8 +131,8 @@ __device__ __forceinline__ void topk_row(const uint32_t (&key)[KPL], int nb, int
   for (int q = 0; q < KPL; ++q) {
     if (q * 32 >= nb) break;
     const int j = q * 32 + lane;
-    const bool is_gt = key[q] > prefix;
-    const bool is_eq = key[q] == prefix;
+    const bool is_gt = key[q] > kth;
+    const bool is_eq = key[q] == kth;
     const uint32_t eq_mask = __ballot_sync(0xffffffffu, is_eq);
     const int eq_rank = eq_seen + __popc(eq_mask & lt_mask);
     const bool sel = is_gt || (is_eq && eq_rank < need_eq);
@@ -216,16 +235,23 @@ __global__ void __launch_bounds__(kThreads, 1) score_topk_kernel(const float* __
     }
   }
 
-  // top-k: one warp per row, the row's keys in registers
+  // top-k: one warp per two rows at a time (r and r + 8 of this warp's share),
+  // the rows' keys in registers
   const int warp = threadIdx.x >> 5;
-  for (int r = warp; r < nrows; r += kThreads / 32) {
-    uint32_t key[KPL];
+  for (int r = warp; r < nrows; r += 2 * (kThreads / 32)) {
+    const int r2 = r + kThreads / 32;
+    const bool two = r2 < nrows;
+    uint32_t key[2][KPL];
 #pragma unroll
     for (int q = 0; q < KPL; ++q) {
       const int j = q * 32 + lane;
-      key[q] = j < nb ? order_key(sc[r * nb + j]) : 0u;
+      key[0][q] = j < nb ? order_key(sc[r * nb + j]) : 0u;
+      key[1][q] = j < nb ? order_key(sc[(two ? r2 : r) * nb + j]) : 0u;
     }
-    topk_row<KPL>(key, nb, topk, idx + (static_cast<size_t>(bh) * nb + r0 + r) * topk, lane);
+    uint32_t kth[2];
+    kth_largest<KPL, 2>(key, topk, kth);
+    compact_row<KPL>(key[0], kth[0], nb, topk, idx + (static_cast<size_t>(bh) * nb + r0 + r) * topk, lane);
+    if (two) compact_row<KPL>(key[1], kth[1], nb, topk, idx + (static_cast<size_t>(bh) * nb + r0 + r2) * topk, lane);
   }
 }
 
