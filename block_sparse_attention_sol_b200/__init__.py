@@ -9,6 +9,10 @@ Functions (same names as the C ABI):
     sol_qk_prologue(q_raw, k_raw, gamma_q, gamma_k, grid, ...)  -> (q, k)
     sol_block_select(q, k, grid, block, topk, ...)              -> idx [, scores]
     sol_sparse_attn_fwd(q, k, v, idx, grid, block, ...)         -> (o, lse)
+    sol_qk_prologue_pool(q_raw, k_raw, gamma_q, gamma_k, grid, block, ...) -> (q, k, qbar, kbar)
+    sol_block_select_pooled(qbar, kbar, grid, block, topk, ...) -> idx [, scores]
+    sol_block_select_pooled_ex(qbar, kbar, grid, block, topk, flags=..., ...) -> (idx, counts) [, scores]
+    sol_sparse_attn_fwd_counts(q, k, v, idx, counts, grid, block, ...) -> (o, lse)
     sol_check_device_status(stream=None)
     sol_selftest_wait_timeout(limit_us, stream=None)
     sol_block_select_workspace_bytes(shape, block)
@@ -23,7 +27,8 @@ import torch
 __all__ = [
     "SolError", "SolShape", "LIB_PATH", "lib",
     "sol_qk_prologue", "sol_block_select", "sol_block_select_workspace_bytes", "sol_sparse_attn_fwd",
-    "sol_qk_prologue_pool", "sol_block_select_pooled",
+    "sol_qk_prologue_pool", "sol_block_select_pooled", "sol_block_select_pooled_ex", "sol_sparse_attn_fwd_counts",
+    "SolSelectOpts", "SOL_SELECT_FORCE_DIAGONAL", "SOL_SELECT_FORCE_FIRST_FRAME", "SOL_SELECT_TOP_P",
     "sol_check_device_status", "sol_selftest_wait_timeout", "sol_status_string", "sol_attention_chain",
     "SOL_OK", "SOL_ERR_INVALID_ARG", "SOL_ERR_UNSUPPORTED", "SOL_ERR_CUDA", "SOL_ERR_TIMEOUT",
 ]
@@ -37,10 +42,16 @@ lib = ctypes.CDLL(LIB_PATH)
 
 SOL_OK, SOL_ERR_INVALID_ARG, SOL_ERR_UNSUPPORTED, SOL_ERR_CUDA, SOL_ERR_TIMEOUT = range(5)
 SOL_F32, SOL_BF16 = 0, 1
+SOL_SELECT_FORCE_DIAGONAL, SOL_SELECT_FORCE_FIRST_FRAME, SOL_SELECT_TOP_P = 1, 2, 4
 
 
 class SolShape(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in ("B", "N", "H", "D", "grid_t", "grid_h", "grid_w")]
+
+
+class SolSelectOpts(ctypes.Structure):
+    _fields_ = [("flags", ctypes.c_uint), ("top_p", ctypes.c_float), ("softmax_scale", ctypes.c_float),
+                ("head_k", ctypes.c_void_p)]
 
 
 class SolError(RuntimeError):
@@ -62,6 +73,10 @@ lib.sol_qk_prologue_pool.restype = _I
 lib.sol_qk_prologue_pool.argtypes = [_P, _P, _P, _P, _P, _P, SolShape, _I, _I, _I, _F, _F, _I, _I, _P, _P, _P]
 lib.sol_block_select_pooled.restype = _I
 lib.sol_block_select_pooled.argtypes = [_P, _P, SolShape, _I, _I, _P, _P, _P]
+lib.sol_block_select_pooled_ex.restype = _I
+lib.sol_block_select_pooled_ex.argtypes = [_P, _P, SolShape, _I, _I, ctypes.POINTER(SolSelectOpts), _P, _P, _P, _P]
+lib.sol_sparse_attn_fwd_counts.restype = _I
+lib.sol_sparse_attn_fwd_counts.argtypes = [_P, _P, _P, _P, _P, SolShape, _I, _I, _F, _I, _P, _P, _P]
 lib.sol_sparse_attn_fwd.restype = _I
 lib.sol_sparse_attn_fwd.argtypes = [_P, _P, _P, _P, SolShape, _I, _I, _F, _I, _P, _P, _P]
 lib.sol_check_device_status.restype = _I
@@ -168,6 +183,36 @@ def sol_block_select_pooled(qbar, kbar, grid, block, topk, idx_out=None, return_
     return (idx_out, scores) if return_scores else idx_out
 
 
+def sol_block_select_pooled_ex(qbar, kbar, grid, block, topk, flags=0, top_p=1.0, softmax_scale=0.0, head_k=None,
+                               idx_out=None, counts_out=None, return_scores=False, stream=None):
+    """Selection variants (forced diagonal / first-frame blocks, top-p, per-head k)
+    from block means.  Returns (idx, counts) (and the scores); rows of idx hold
+    their count of ascending ids, then -1."""
+    _cuda(qbar, "qbar"), _cuda(kbar, "kbar")
+    if qbar.dtype != torch.float32 or kbar.dtype != torch.float32:
+        raise TypeError("qbar and kbar must be float32")
+    B, H, nb, D = qbar.shape
+    N = int(grid[0]) * int(grid[1]) * int(grid[2])
+    s = SolShape(B, N, H, D, int(grid[0]), int(grid[1]), int(grid[2]))
+    if head_k is not None:
+        _cuda(head_k, "head_k")
+        if head_k.dtype != torch.int32 or head_k.numel() != H:
+            raise ValueError("head_k must be int32 [H]")
+    if idx_out is None:
+        idx_out = torch.empty((B, H, nb, topk), dtype=torch.int32, device=qbar.device)
+    if counts_out is None:
+        counts_out = torch.empty((B, H, nb), dtype=torch.int32, device=qbar.device)
+    scores = torch.empty((B, H, nb, nb), dtype=torch.float32, device=qbar.device) if return_scores else None
+    opts = SolSelectOpts(int(flags), float(top_p), float(softmax_scale),
+                         head_k.data_ptr() if head_k is not None else None)
+    st = lib.sol_block_select_pooled_ex(qbar.data_ptr(), kbar.data_ptr(), s, int(block), int(topk),
+                                        ctypes.byref(opts), _cuda(idx_out, "idx_out").data_ptr(),
+                                        _cuda(counts_out, "counts_out").data_ptr(),
+                                        scores.data_ptr() if scores is not None else None, _stream_handle(stream))
+    _check(st, "sol_block_select_pooled_ex")
+    return (idx_out, counts_out, scores) if return_scores else (idx_out, counts_out)
+
+
 def sol_block_select_workspace_bytes(shape: SolShape, block: int) -> int:
     return int(lib.sol_block_select_workspace_bytes(shape, int(block)))
 
@@ -206,6 +251,22 @@ def sol_sparse_attn_fwd(q, k, v, idx, grid, block, softmax_scale=0.0, o=None, ls
                                  float(softmax_scale), _dtype_code(q), o.data_ptr(), lse.data_ptr(),
                                  _stream_handle(stream))
     _check(st, "sol_sparse_attn_fwd")
+    return o, lse
+
+
+def sol_sparse_attn_fwd_counts(q, k, v, idx, counts, grid, block, softmax_scale=0.0, o=None, lse=None, stream=None):
+    """sol_sparse_attn_fwd where row (b, h, i) uses only its first counts[b, h, i] ids."""
+    _cuda(q, "q"), _cuda(k, "k"), _cuda(v, "v"), _cuda(idx, "idx"), _cuda(counts, "counts")
+    if idx.dtype != torch.int32 or counts.dtype != torch.int32:
+        raise TypeError("idx and counts must be int32")
+    s = _shape(q, grid)
+    topk = idx.shape[-1]
+    o = torch.empty_like(q) if o is None else _cuda(o, "o")
+    lse = torch.empty((s.B, s.H, s.N), dtype=torch.float32, device=q.device) if lse is None else _cuda(lse, "lse")
+    st = lib.sol_sparse_attn_fwd_counts(q.data_ptr(), k.data_ptr(), v.data_ptr(), idx.data_ptr(), counts.data_ptr(),
+                                        s, int(block), int(topk), float(softmax_scale), _dtype_code(q), o.data_ptr(),
+                                        lse.data_ptr(), _stream_handle(stream))
+    _check(st, "sol_sparse_attn_fwd_counts")
     return o, lse
 
 

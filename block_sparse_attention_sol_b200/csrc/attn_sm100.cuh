@@ -69,6 +69,7 @@ struct __align__(1024) Smem {
 struct Params {
   const __nv_bfloat16* q; // [B, N, H, D]
   const int32_t* idx;     // [B, H, nb, topk]
+  const int32_t* counts;  // [B, H, nb] blocks used per row (clamped to [1, topk]), or null: topk
   __nv_bfloat16* o;       // [B, N, H, D]
   float* lse;             // [B, H, N]
   int B, N, H, nb, topk;
@@ -84,6 +85,11 @@ enum : unsigned { kSiteQEmpty = 1, kSiteSlotFree, kSiteQFull, kSiteSlotFull, kSi
 // channels = 32 bytes per step, the second 64-channel box 16 KB further.
 __device__ __forceinline__ constexpr uint32_t kstep_off(int kk) {
   return static_cast<uint32_t>(((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4);
+}
+
+// Key blocks of tile t (row t of idx in [B, H, nb] order); every role reads the same value.
+__device__ __forceinline__ int tile_steps(const Params& p, int t) {
+  return p.counts == nullptr ? p.topk : min(max(__ldg(p.counts + t), 1), p.topk);
 }
 
 __device__ __forceinline__ void decode_tile(const Params& p, int t, int& b, int& h, int& qb) {
@@ -133,11 +139,12 @@ sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
         int b, h, qb;
         decode_tile(p, t, b, h, qb);
         const int32_t* list = p.idx + (static_cast<size_t>(b * p.H + h) * p.nb + qb) * p.topk;
-        // slot s of the tile: K_s (s < topk) and V_{s-2} (s >= 2), in the order the MMA issuer uses them
-        for (int s = 0; s < p.topk + 2; ++s, ++sq) {
+        const int kt = tile_steps(p, t);
+        // slot s of the tile: K_s (s < kt) and V_{s-2} (s >= 2), in the order the MMA issuer uses them
+        for (int s = 0; s < kt + 2; ++s, ++sq) {
           const uint32_t st = sq % kSlots, use = sq / kSlots;
           if (use > 0 && !(ok = mbar_wait(&sm.slot_done[st], (use - 1) & 1, abort_flag, kSiteSlotFree))) break;
-          const bool has_k = s < p.topk, has_v = s >= 2;
+          const bool has_k = s < kt, has_v = s >= 2;
           mbar_arrive_expect_tx(&sm.kv_full[st], (has_k ? kTileBytes : 0) + (has_v ? kTileBytes : 0));
           if (has_k) {
             const int blk = __ldg(list + s);
@@ -187,17 +194,18 @@ sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
       };
       for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x, ++it) {
         if (!(ok = mbar_wait(&sm.q_full, it & 1, abort_flag, kSiteQFull))) break;
-        // slots 0 and 1 of the tile: K_0 and K_1 (slot 1 is empty when topk = 1)
+        const int kt = tile_steps(p, t);
+        // slots 0 and 1 of the tile: K_0 and K_1 (slot 1 is empty when kt = 1)
         for (int s = 0; s < 2 && ok; ++s) {
           const uint32_t sl = sq + s, st = sl % kSlots;
           if (!(ok = mbar_wait(&sm.kv_full[st], (sl / kSlots) & 1, abort_flag, kSiteSlotFull))) break;
           tc_fence_after();
-          if (s < p.topk) mma_s(g + s, st);
+          if (s < kt) mma_s(g + s, st);
           tc_commit(&sm.slot_done[st]);
         }
         if (!ok) break;
-        if (p.topk <= 2) tc_commit(&sm.q_empty);   // every S MMA of this tile has been issued
-        for (int j = 0; j < p.topk; ++j) {
+        if (kt <= 2) tc_commit(&sm.q_empty);   // every S MMA of this tile has been issued
+        for (int j = 0; j < kt; ++j) {
           const uint32_t gg = g + j, sl = sq + j + 2, st = sl % kSlots;
           if (!(ok = mbar_wait(&sm.p_full, gg & 1, abort_flag, kSitePFull))) break;
           if (j == 0 && it > 0 && !(ok = mbar_wait(&sm.o_free, (it - 1) & 1, abort_flag, kSiteOFree))) break;
@@ -209,12 +217,12 @@ sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
             mma_ts(o_tm, p_tm + kk * 8, vd + static_cast<uint32_t>(kk * 128), kIdescPV,
                    (j > 0 || kk > 0) ? 1u : 0u);
           tc_commit(&sm.pv_done);
-          if (j + 2 < p.topk) mma_s(gg + 2, st);
+          if (j + 2 < kt) mma_s(gg + 2, st);
           tc_commit(&sm.slot_done[st]);
-          if (j + 3 == p.topk) tc_commit(&sm.q_empty);
+          if (j + 3 == kt) tc_commit(&sm.q_empty);
         }
-        g += p.topk;
-        sq += p.topk + 2;
+        g += kt;
+        sq += kt + 2;
       }
       // Drain: every MMA issued must complete before TMEM is released.
       tc_commit(&sm.drain);
@@ -244,6 +252,7 @@ sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
       int b, h, qb;
       decode_tile(p, t, b, h, qb);
       const int32_t* list = p.idx + (static_cast<size_t>(b * p.H + h) * p.nb + qb) * p.topk;
+      const int kt = tile_steps(p, t);
       // ---- Q into TMEM (A operand of the S MMAs: lane = row, 2 bf16 per column).
       // The two warps of a quadrant write channels [64 half, 64 half + 64) of its 32 rows.
       if (it > 0) {
@@ -275,10 +284,10 @@ sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
       float m0 = -INFINITY, m1 = -INFINITY;   // running max per row, log2 units (stale by < 2^8)
       float l0 = 0.f, l1 = 0.f;               // this thread's part of the running sums
       int blk = __ldg(list);
-      for (int j = 0; j < p.topk; ++j) {
+      for (int j = 0; j < kt; ++j) {
         const uint32_t gg = g + j;
         const uint32_t buf = gg & 1;
-        const int blk_next = (j + 1 < p.topk) ? __ldg(list + j + 1) : 0;
+        const int blk_next = (j + 1 < kt) ? __ldg(list + j + 1) : 0;
         const uint32_t sl = sq + j;   // slot of K_j: its slot_done also means S_j is complete
         ok = mbar_wait(&sm.slot_done[sl % kSlots], (sl / kSlots) & 1, abort_flag, kSiteSDone);
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
@@ -384,7 +393,7 @@ sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
       if (!ok) break;
       // epilogue: O / l and LSE
       {
-        ok = mbar_wait(&sm.pv_done, (g + p.topk - 1) & 1, abort_flag, kSitePvDone);
+        ok = mbar_wait(&sm.pv_done, (g + kt - 1) & 1, abort_flag, kSitePvDone);
       }
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
@@ -424,8 +433,8 @@ sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
                 ((u ? m1 : m0) + __log2f(u ? l1 : l0)) * 0.69314718055994531f;
         }
       }
-      g += p.topk;
-      sq += p.topk + 2;
+      g += kt;
+      sq += kt + 2;
     }
   }
 

@@ -18,6 +18,7 @@
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
+#include <cmath>
 
 namespace sol {
 namespace select {
@@ -143,23 +144,41 @@ __device__ __forceinline__ void compact_row(const uint32_t (&key)[KPL], uint32_t
   }
 }
 
+// Selection variants, all optional (zero / null: plain top-k):
+//  - kForceDiagonal keeps the query's own key block, kForceFirstFrame the key
+//    blocks 0 .. n_first - 1 (those holding tokens of the first latent frame),
+//    ahead of every scored block (forced blocks beyond the row's k: lowest ids);
+//  - head_k[h] (device, clamped to [1, topk]) replaces topk for head h;
+//  - kTopP keeps, instead of a fixed k, the shortest prefix of the row's order
+//    (forced blocks first, then descending score, ties to the lower id) whose
+//    softmax mass, softmax_j(scale s_ij) over all key blocks, reaches top_p;
+//    at least the forced blocks and one block, at most the row's k.
+//  A row's ids beyond its count are set to -1; counts (nullable) receives the count.
+enum : unsigned { kForceDiagonal = 1u, kForceFirstFrame = 2u, kTopP = 4u };
+
+struct SelectArgs {
+  int32_t* idx;            // [B, H, nb, topk]
+  float* scores;           // nullable [B, H, nb, nb]
+  int32_t* counts;         // nullable [B, H, nb]
+  const int32_t* head_k;   // nullable [H]
+  int nb, topk, H;
+  unsigned flags;
+  int n_first;
+  float top_p;             // in (0, 1] with kTopP
+  float scale_log2;        // softmax scale * log2(e) with kTopP
+};
+
 // Dynamic shared memory: qs[rows][D+4] | ks[kKeys][D+4] | sc[rows][nb].  The 4-float row
 // padding puts the 16-byte loads of 8 consecutive rows on distinct banks.
-// grid (ceil(nb / (8 RPW)), B * H).  KPL = keys per lane in the top-k, nb <= 32 * KPL.
-template <int D, int RPW, int KPL>
-__global__ void __launch_bounds__(kThreads, 1) score_topk_kernel(const float* __restrict__ qbar,
-                                                                 const float* __restrict__ kbar,
-                                                                 int32_t* __restrict__ idx,
-                                                                 float* __restrict__ scores_out, int nb, int topk) {
-  extern __shared__ float smem[];
+// Scores of rows r0 .. r0 + nrows - 1 of (b, h) = bh against all key blocks, left in sc.
+template <int D, int RPW>
+__device__ __forceinline__ void score_rows(const float* __restrict__ qbar, const float* __restrict__ kbar, float* smem,
+                                           int bh, int r0, int nrows, int nb, float* __restrict__ scores_out) {
   constexpr int P = D + 4;
   constexpr int kRows = 8 * RPW;
   float* qs = smem;
   float* ks = qs + kRows * P;
   float* sc = ks + kKeys * P;
-  const int bh = blockIdx.y;
-  const int r0 = blockIdx.x * kRows;
-  const int nrows = min(kRows, nb - r0);
   const float* qb = qbar + static_cast<size_t>(bh) * nb * D;
   const float* kb = kbar + static_cast<size_t>(bh) * nb * D;
 
@@ -234,24 +253,152 @@ __global__ void __launch_bounds__(kThreads, 1) score_topk_kernel(const float* __
       scores_out[(static_cast<size_t>(bh) * nb + r0 + r) * nb + j] = sc[r * nb + j];
     }
   }
+}
+
+// Order-preserving key of score j of a row, or the largest key for a forced block
+// (order_key of a finite score never reaches it), 0 for padding j >= nb.
+__device__ __forceinline__ uint32_t select_key(const float* row_scores, int j, int i, const SelectArgs& a) {
+  if (j >= a.nb) return 0u;
+  const bool forced = ((a.flags & kForceDiagonal) && j == i) || ((a.flags & kForceFirstFrame) && j < a.n_first);
+  return forced ? 0xffffffffu : order_key(row_scores[j]);
+}
+
+// Writes the row's ids beyond its count as -1 and the count itself.
+__device__ __forceinline__ void finish_row(const SelectArgs& a, size_t row, int count, int lane) {
+  for (int e = count + lane; e < a.topk; e += 32) a.idx[row * a.topk + e] = -1;
+  if (a.counts != nullptr && lane == 0) a.counts[row] = count;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+  // xor butterfly: every lane ends with the same sum, added in the same order
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Softmax mass of the keys >= t (each lane adds its own in slot order, then the warp sums).
+template <int KPL>
+__device__ __forceinline__ float mass_at_least(const uint32_t (&key)[KPL], const float (&e)[KPL], uint32_t t) {
+  float m = 0.f;
+#pragma unroll
+  for (int q = 0; q < KPL; ++q) m += key[q] >= t ? e[q] : 0.f;
+  return warp_sum(m);
+}
+
+// grid (ceil(nb / (8 RPW)), B * H).  KPL = keys per lane in the top-k, nb <= 32 * KPL.
+template <int D, int RPW, int KPL>
+__global__ void __launch_bounds__(kThreads, 1) score_topk_kernel(const float* __restrict__ qbar,
+                                                                 const float* __restrict__ kbar, SelectArgs a) {
+  extern __shared__ float smem[];
+  constexpr int kRows = 8 * RPW;
+  const int nb = a.nb;
+  const int bh = blockIdx.y;
+  const int r0 = blockIdx.x * kRows;
+  const int nrows = min(kRows, nb - r0);
+  score_rows<D, RPW>(qbar, kbar, smem, bh, r0, nrows, nb, a.scores);
+  const float* sc = smem + (kRows + kKeys) * (D + 4);
 
   // top-k: one warp per two rows at a time (r and r + 8 of this warp's share),
   // the rows' keys in registers
+  const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
+  const int kr = a.head_k == nullptr ? a.topk : min(max(__ldg(a.head_k + bh % a.H), 1), a.topk);
   for (int r = warp; r < nrows; r += 2 * (kThreads / 32)) {
     const int r2 = r + kThreads / 32;
     const bool two = r2 < nrows;
+    const int rr[2] = {r, two ? r2 : r};
     uint32_t key[2][KPL];
+#pragma unroll
+    for (int q = 0; q < KPL; ++q)
+#pragma unroll
+      for (int u = 0; u < 2; ++u) key[u][q] = select_key(sc + rr[u] * nb, q * 32 + lane, r0 + rr[u], a);
+    uint32_t kth[2];
+    kth_largest<KPL, 2>(key, kr, kth);
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      if (u == 1 && !two) break;
+      const size_t row = static_cast<size_t>(bh) * nb + r0 + rr[u];
+      compact_row<KPL>(key[u], kth[u], nb, kr, a.idx + row * a.topk, lane);
+      finish_row(a, row, kr, lane);
+    }
+  }
+}
+
+// Top-p selection (kTopP): one warp per row, keys and softmax terms in registers.
+// The cut is found as the largest key T whose mass(key >= T) reaches top_p times
+// the row's total, by the same most-significant-bit-first search as the top-k;
+// blocks tied at T are then taken in id order until the mass is reached.
+template <int D, int RPW, int KPL>
+__global__ void __launch_bounds__(kThreads, 1) score_topp_kernel(const float* __restrict__ qbar,
+                                                                 const float* __restrict__ kbar, SelectArgs a) {
+  extern __shared__ float smem[];
+  constexpr int kRows = 8 * RPW;
+  const int nb = a.nb;
+  const int bh = blockIdx.y;
+  const int r0 = blockIdx.x * kRows;
+  const int nrows = min(kRows, nb - r0);
+  score_rows<D, RPW>(qbar, kbar, smem, bh, r0, nrows, nb, a.scores);
+  const float* sc = smem + (kRows + kKeys) * (D + 4);
+
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int kcap = a.head_k == nullptr ? a.topk : min(max(__ldg(a.head_k + bh % a.H), 1), a.topk);
+  for (int r = warp; r < nrows; r += kThreads / 32) {
+    const float* row_sc = sc + r * nb;
+    float mx = -INFINITY;
+#pragma unroll
+    for (int q = 0; q < KPL; ++q)
+      if (q * 32 + lane < nb) mx = fmaxf(mx, row_sc[q * 32 + lane]);
+    mx = warp_max(mx);
+    uint32_t key[KPL];
+    float e[KPL];
+    uint32_t nf = 0;
 #pragma unroll
     for (int q = 0; q < KPL; ++q) {
       const int j = q * 32 + lane;
-      key[0][q] = j < nb ? order_key(sc[r * nb + j]) : 0u;
-      key[1][q] = j < nb ? order_key(sc[(two ? r2 : r) * nb + j]) : 0u;
+      key[q] = select_key(row_sc, j, r0 + r, a);
+      e[q] = j < nb ? exp2f((row_sc[j] - mx) * a.scale_log2) : 0.f;
+      nf += key[q] == 0xffffffffu ? 1u : 0u;
     }
-    uint32_t kth[2];
-    kth_largest<KPL, 2>(key, topk, kth);
-    compact_row<KPL>(key[0], kth[0], nb, topk, idx + (static_cast<size_t>(bh) * nb + r0 + r) * topk, lane);
-    if (two) compact_row<KPL>(key[1], kth[1], nb, topk, idx + (static_cast<size_t>(bh) * nb + r0 + r2) * topk, lane);
+    const int n_forced = static_cast<int>(__reduce_add_sync(0xffffffffu, nf));
+    const float target = a.top_p * mass_at_least<KPL>(key, e, 0u);
+    uint32_t t = 0u;
+#pragma unroll 1
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t cand = t | (1u << bit);
+      if (mass_at_least<KPL>(key, e, cand) >= target) t = cand;
+    }
+    int count = n_forced;
+    if (t != 0xffffffffu) {
+      uint32_t gt = 0, eq = 0;
+      float et = 0.f;
+#pragma unroll
+      for (int q = 0; q < KPL; ++q) {
+        gt += key[q] > t ? 1u : 0u;
+        eq += key[q] == t ? 1u : 0u;
+        if (key[q] == t) et = e[q];   // tied keys are equal scores: equal terms
+      }
+      const int n_gt = static_cast<int>(__reduce_add_sync(0xffffffffu, gt));
+      const int n_eq = static_cast<int>(__reduce_add_sync(0xffffffffu, eq));
+      et = warp_max(et);
+      const float need = target - mass_at_least<KPL>(key, e, t + 1u);
+      const float take = et > 0.f ? fminf(ceilf(need / et), static_cast<float>(n_eq)) : static_cast<float>(n_eq);
+      count = max(count, n_gt + max(static_cast<int>(take), 1));
+    }
+    count = min(max(count, 1), kcap);
+    uint32_t keys1[1][KPL];
+#pragma unroll
+    for (int q = 0; q < KPL; ++q) keys1[0][q] = key[q];
+    uint32_t kth[1];
+    kth_largest<KPL, 1>(keys1, count, kth);
+    const size_t row = static_cast<size_t>(bh) * nb + r0 + r;
+    compact_row<KPL>(keys1[0], kth[0], nb, count, a.idx + row * a.topk, lane);
+    finish_row(a, row, count, lane);
   }
 }
 

@@ -49,7 +49,7 @@ int num_blocks(int N, int block) { return (N + block - 1) / block; }
 struct DeviceInfo {
   int sm_count = 0;
   bool attn_attr = false, attn_pp_attr = false;
-  bool select_attr[16] = {};   // score_topk_kernel instantiations with the shared-memory opt-in set
+  bool select_attr[32] = {};   // score_topk / score_topp_kernel instantiations with the shared-memory opt-in set
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -136,41 +136,54 @@ sol_status plan_scores(const sol_shape& s, int nb, ScorePlan* plan) {
   return SOL_OK;
 }
 
-// Launches score_topk_kernel<D, RPW, KPL> for the runtime choices (shared-memory
-// opt-in set once per device and instantiation).
+// Launches score_topk_kernel<D, RPW, KPL> (or score_topp_kernel with kTopP) for the
+// runtime choices (shared-memory opt-in set once per device and instantiation).
 template <int D, int RPW, int KPL>
 sol_status launch_score_topk_t(DeviceInfo* di, dim3 grid, size_t smem, cudaStream_t stream, const float* qbar,
-                               const float* kbar, int32_t* idx, float* scores, int nb, int topk) {
-  constexpr int slot = (D == 128 ? 8 : 0) + (RPW == 4 ? 4 : 0) + (KPL == 8 ? 0 : KPL == 16 ? 1 : KPL == 32 ? 2 : 3);
+                               const float* kbar, const sol::select::SelectArgs& a) {
+  const bool topp = (a.flags & sol::select::kTopP) != 0u;
+  auto kernel = topp ? sol::select::score_topp_kernel<D, RPW, KPL> : sol::select::score_topk_kernel<D, RPW, KPL>;
+  const int slot = (topp ? 16 : 0) + (D == 128 ? 8 : 0) + (RPW == 4 ? 4 : 0) +
+                   (KPL == 8 ? 0 : KPL == 16 ? 1 : KPL == 32 ? 2 : 3);
   if (!di->select_attr[slot]) {
-    if (cudaFuncSetAttribute(sol::select::score_topk_kernel<D, RPW, KPL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kMaxSmemPerBlock)) != cudaSuccess)
       return SOL_ERR_CUDA;
     di->select_attr[slot] = true;
   }
-  sol::select::score_topk_kernel<D, RPW, KPL><<<grid, sol::select::kThreads, smem, stream>>>(qbar, kbar, idx, scores,
-                                                                                            nb, topk);
+  kernel<<<grid, sol::select::kThreads, smem, stream>>>(qbar, kbar, a);
   return launch_status();
 }
 
 template <int D, int RPW>
 sol_status launch_score_topk_k(DeviceInfo* di, int kpl, dim3 grid, size_t smem, cudaStream_t stream,
-                               const float* qbar, const float* kbar, int32_t* idx, float* scores, int nb, int topk) {
+                               const float* qbar, const float* kbar, const sol::select::SelectArgs& a) {
   switch (kpl) {
-    case 8: return launch_score_topk_t<D, RPW, 8>(di, grid, smem, stream, qbar, kbar, idx, scores, nb, topk);
-    case 16: return launch_score_topk_t<D, RPW, 16>(di, grid, smem, stream, qbar, kbar, idx, scores, nb, topk);
-    case 32: return launch_score_topk_t<D, RPW, 32>(di, grid, smem, stream, qbar, kbar, idx, scores, nb, topk);
-    default: return launch_score_topk_t<D, RPW, 64>(di, grid, smem, stream, qbar, kbar, idx, scores, nb, topk);
+    case 8: return launch_score_topk_t<D, RPW, 8>(di, grid, smem, stream, qbar, kbar, a);
+    case 16: return launch_score_topk_t<D, RPW, 16>(di, grid, smem, stream, qbar, kbar, a);
+    case 32: return launch_score_topk_t<D, RPW, 32>(di, grid, smem, stream, qbar, kbar, a);
+    default: return launch_score_topk_t<D, RPW, 64>(di, grid, smem, stream, qbar, kbar, a);
   }
 }
 
-sol_status launch_score_topk(DeviceInfo* di, int D, int rpw, int kpl, dim3 grid, size_t smem, cudaStream_t stream,
-                             const float* qbar, const float* kbar, int32_t* idx, float* scores, int nb, int topk) {
+sol_status launch_score_topk(DeviceInfo* di, int D, const ScorePlan& plan, cudaStream_t stream, const float* qbar,
+                             const float* kbar, const sol::select::SelectArgs& a) {
   if (D == 128)
-    return rpw == 4 ? launch_score_topk_k<128, 4>(di, kpl, grid, smem, stream, qbar, kbar, idx, scores, nb, topk)
-                    : launch_score_topk_k<128, 2>(di, kpl, grid, smem, stream, qbar, kbar, idx, scores, nb, topk);
-  return rpw == 4 ? launch_score_topk_k<64, 4>(di, kpl, grid, smem, stream, qbar, kbar, idx, scores, nb, topk)
-                  : launch_score_topk_k<64, 2>(di, kpl, grid, smem, stream, qbar, kbar, idx, scores, nb, topk);
+    return plan.rpw == 4 ? launch_score_topk_k<128, 4>(di, plan.kpl, plan.grid, plan.smem, stream, qbar, kbar, a)
+                         : launch_score_topk_k<128, 2>(di, plan.kpl, plan.grid, plan.smem, stream, qbar, kbar, a);
+  return plan.rpw == 4 ? launch_score_topk_k<64, 4>(di, plan.kpl, plan.grid, plan.smem, stream, qbar, kbar, a)
+                       : launch_score_topk_k<64, 2>(di, plan.kpl, plan.grid, plan.smem, stream, qbar, kbar, a);
+}
+
+// Plain top-k arguments: no forced blocks, one k for every head, no counts.
+sol::select::SelectArgs plain_select(const sol_shape& s, int nb, int topk, int32_t* idx, float* scores) {
+  sol::select::SelectArgs a{};
+  a.idx = idx;
+  a.scores = scores;
+  a.nb = nb;
+  a.topk = topk;
+  a.H = s.H;
+  return a;
 }
 
 }  // namespace
@@ -208,6 +221,13 @@ sol_status prologue_params(const void* q_raw, const void* k_raw, void* q_out, vo
   return SOL_OK;
 }
 
+}  // namespace
+
+namespace {
+// Attention with optional per-row block counts (both attention entry points).
+sol_status sparse_attn_impl(const void* q, const void* k, const void* v, const int32_t* idx, const int32_t* counts,
+                            sol_shape s, int block, int topk, float softmax_scale, sol_dtype dt, void* o, float* lse,
+                            cudaStream_t stream);
 }  // namespace
 
 extern "C" {
@@ -319,8 +339,7 @@ sol_status sol_block_select(const void* q, const void* k, sol_shape s, int block
                                                                   static_cast<const float*>(k), qbar, kbar, s.N, s.H,
                                                                   s.D, block, nb);
   if (sol_status st = launch_status()) return st;
-  return launch_score_topk(di, s.D, plan.rpw, plan.kpl, plan.grid, plan.smem, stream, qbar, kbar, idx_out,
-                           scores_out, nb, topk);
+  return launch_score_topk(di, s.D, plan, stream, qbar, kbar, plain_select(s, nb, topk, idx_out, scores_out));
 }
 
 sol_status sol_block_select_pooled(const float* qbar, const float* kbar, sol_shape s, int block, int topk,
@@ -335,13 +354,62 @@ sol_status sol_block_select_pooled(const float* qbar, const float* kbar, sol_sha
   if (sol_status st = plan_scores(s, nb, &plan)) return st;
   DeviceInfo* di = nullptr;
   if (sol_status st = device_info(&di)) return st;
-  return launch_score_topk(di, s.D, plan.rpw, plan.kpl, plan.grid, plan.smem, stream, qbar, kbar, idx_out,
-                           scores_out, nb, topk);
+  return launch_score_topk(di, s.D, plan, stream, qbar, kbar, plain_select(s, nb, topk, idx_out, scores_out));
+}
+
+sol_status sol_block_select_pooled_ex(const float* qbar, const float* kbar, sol_shape s, int block, int topk,
+                                      const sol_select_opts* opts, int32_t* idx_out, int32_t* counts_out,
+                                      float* scores_out, cudaStream_t stream) {
+  if (!qbar || !kbar || !idx_out || !counts_out || !opts) return SOL_ERR_INVALID_ARG;
+  if (!aligned16(qbar) || !aligned16(kbar) || !aligned16(idx_out) || !aligned16(counts_out))
+    return SOL_ERR_INVALID_ARG;
+  if (scores_out && !aligned16(scores_out)) return SOL_ERR_INVALID_ARG;
+  if (!shape_ok(s) || block <= 0) return SOL_ERR_INVALID_ARG;
+  const unsigned known = SOL_SELECT_FORCE_DIAGONAL | SOL_SELECT_FORCE_FIRST_FRAME | SOL_SELECT_TOP_P;
+  if (opts->flags & ~known) return SOL_ERR_INVALID_ARG;
+  const bool topp = (opts->flags & SOL_SELECT_TOP_P) != 0u;
+  if (topp && !(opts->top_p > 0.f && opts->top_p <= 1.f)) return SOL_ERR_INVALID_ARG;
+  if (topp && !std::isfinite(opts->softmax_scale)) return SOL_ERR_INVALID_ARG;
+  const int nb = num_blocks(s.N, block);
+  if (topk < 1 || topk > nb) return SOL_ERR_INVALID_ARG;
+  ScorePlan plan;
+  if (sol_status st = plan_scores(s, nb, &plan)) return st;
+  DeviceInfo* di = nullptr;
+  if (sol_status st = device_info(&di)) return st;
+  sol::select::SelectArgs a = plain_select(s, nb, topk, idx_out, scores_out);
+  a.counts = counts_out;
+  a.head_k = opts->head_k;
+  a.flags = (opts->flags & SOL_SELECT_FORCE_DIAGONAL ? sol::select::kForceDiagonal : 0u) |
+            (opts->flags & SOL_SELECT_FORCE_FIRST_FRAME ? sol::select::kForceFirstFrame : 0u) |
+            (topp ? sol::select::kTopP : 0u);
+  // blocks holding a token of frame t = 0: tokens 0 .. grid_h * grid_w - 1 in raster order
+  a.n_first = num_blocks(s.grid_h * s.grid_w, block);
+  a.top_p = opts->top_p;
+  const float scale = opts->softmax_scale > 0.f ? opts->softmax_scale : 1.0f / std::sqrt(static_cast<float>(s.D));
+  a.scale_log2 = scale * 1.4426950408889634f;   // log2(e)
+  return launch_score_topk(di, s.D, plan, stream, qbar, kbar, a);
 }
 
 sol_status sol_sparse_attn_fwd(const void* q, const void* k, const void* v, const int32_t* idx, sol_shape s,
                                int block, int topk, float softmax_scale, sol_dtype dt, void* o, float* lse,
                                cudaStream_t stream) {
+  return sparse_attn_impl(q, k, v, idx, nullptr, s, block, topk, softmax_scale, dt, o, lse, stream);
+}
+
+sol_status sol_sparse_attn_fwd_counts(const void* q, const void* k, const void* v, const int32_t* idx,
+                                      const int32_t* counts, sol_shape s, int block, int topk, float softmax_scale,
+                                      sol_dtype dt, void* o, float* lse, cudaStream_t stream) {
+  if (!counts) return SOL_ERR_INVALID_ARG;
+  return sparse_attn_impl(q, k, v, idx, counts, s, block, topk, softmax_scale, dt, o, lse, stream);
+}
+
+}  // extern "C"
+
+namespace {
+
+sol_status sparse_attn_impl(const void* q, const void* k, const void* v, const int32_t* idx, const int32_t* counts,
+                            sol_shape s, int block, int topk, float softmax_scale, sol_dtype dt, void* o, float* lse,
+                            cudaStream_t stream) {
   if (!q || !k || !v || !idx || !o || !lse) return SOL_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(idx) || !aligned16(lse))
     return SOL_ERR_INVALID_ARG;
@@ -362,11 +430,11 @@ sol_status sol_sparse_attn_fwd(const void* q, const void* k, const void* v, cons
     if (grid > 0x7fffffffll) return SOL_ERR_UNSUPPORTED;
     if (s.D == 128)
       sol::attnf32::sparse_attn_fwd_f32_kernel<128><<<static_cast<int>(grid), sol::attnf32::kWarps * 32, 0, stream>>>(
-          static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v), idx,
+          static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v), idx, counts,
           static_cast<float*>(o), lse, s.B, s.N, s.H, block, nb, topk, scale);
     else
       sol::attnf32::sparse_attn_fwd_f32_kernel<64><<<static_cast<int>(grid), sol::attnf32::kWarps * 32, 0, stream>>>(
-          static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v), idx,
+          static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v), idx, counts,
           static_cast<float*>(o), lse, s.B, s.N, s.H, block, nb, topk, scale);
     return launch_status();
   }
@@ -414,6 +482,7 @@ sol_status sol_sparse_attn_fwd(const void* q, const void* k, const void* v, cons
   sol::attn100::Params p;
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.idx = idx;
+  p.counts = counts;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   p.B = s.B; p.N = s.N; p.H = s.H; p.nb = nb; p.topk = topk;
@@ -423,6 +492,10 @@ sol_status sol_sparse_attn_fwd(const void* q, const void* k, const void* v, cons
   sol::attn100::sparse_attn_fwd_kernel<<<grid, sol::attn100::kThreads, smem, stream>>>(tk, tv, p);
   return launch_status();
 }
+
+}  // namespace
+
+extern "C" {
 
 // ---------------------------------------------------------------- no-alloc select
 // Scratch for sol_block_select_noalloc: one array per device, shared by every

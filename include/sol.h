@@ -133,6 +133,56 @@ sol_status sol_block_select_pooled(const float* qbar, const float* kbar, sol_sha
                                    int32_t* idx_out, float* scores_out, cudaStream_t stream);
 
 /*
+ * Selection variants -- the per-query choices the pages leave open (Sol-Attn
+ * "decides per query" which parts of the attention matter: ai-feiten.nl,
+ * "Videomodel MiniMax-H3 rendert sneller dan afspelen", section "Waar de
+ * snelheidswinst vandaan komt"; the rules below are this library's readings).
+ *
+ * flags:
+ *  SOL_SELECT_FORCE_DIAGONAL    every query block keeps its own key block i.
+ *  SOL_SELECT_FORCE_FIRST_FRAME every query block keeps the key blocks that hold
+ *                               tokens of frame t = 0: ids 0 .. ceil(grid_h *
+ *                               grid_w / block) - 1.
+ *  SOL_SELECT_TOP_P             the row keeps a mass-based count instead of a
+ *                               fixed one (below).
+ * A row's order is: forced blocks (ascending id), then the other blocks by
+ * descending score, exact ties to the lower id.  A row keeps a prefix of that
+ * order of length c, written in ascending id:
+ *  - without TOP_P, c = k_h;
+ *  - with TOP_P, c = min(k_h, max(forced blocks in the row, 1, the shortest
+ *    prefix length whose mass reaches top_p)), where the mass of block j is
+ *    softmax_j(scale * s[b,h,i,j]) over all nb key blocks and scale =
+ *    softmax_scale (<= 0: 1/sqrt(D)).
+ * k_h = topk, or head_k[h] clamped to [1, topk] when head_k (device int32 [H])
+ * is not NULL.  Forced blocks beyond k_h: the lowest ids are kept.
+ */
+#define SOL_SELECT_FORCE_DIAGONAL 1u
+#define SOL_SELECT_FORCE_FIRST_FRAME 2u
+#define SOL_SELECT_TOP_P 4u
+typedef struct {
+  unsigned flags;          /* OR of SOL_SELECT_* (0: plain top-k)           */
+  float top_p;             /* in (0, 1], read with SOL_SELECT_TOP_P         */
+  float softmax_scale;     /* top-p softmax scale, <= 0: 1/sqrt(D)          */
+  const int32_t* head_k;   /* NULL, or device int32 [H] per-head k          */
+} sol_select_opts;
+
+/*
+ * sol_block_select_pooled_ex -- sol_block_select_pooled with the variants above.
+ *
+ * idx_out    : int32 [B, H, nb, topk]; row (b,h,i) holds its c ids in ascending
+ *              order, then topk - c entries of -1.
+ * counts_out : int32 [B, H, nb], c per row (required: sol_sparse_attn_fwd_counts
+ *              reads it).
+ * opts       : host pointer, read during the call.  Unknown flags, top_p outside
+ *              (0, 1] with TOP_P, or a non-finite softmax_scale: SOL_ERR_INVALID_ARG.
+ * With opts->flags == 0 and head_k NULL, idx_out equals sol_block_select_pooled's
+ * and every count is topk.  Other arguments and limits as sol_block_select_pooled.
+ */
+sol_status sol_block_select_pooled_ex(const float* qbar, const float* kbar, sol_shape s, int block, int topk,
+                                      const sol_select_opts* opts, int32_t* idx_out, int32_t* counts_out,
+                                      float* scores_out, cudaStream_t stream);
+
+/*
  * sol_sparse_attn_fwd -- Sol-Attn block-sparse attention forward
  * (ai-feiten.nl, same section: attention restricted, per query, to the parts
  * that matter).
@@ -151,6 +201,20 @@ sol_status sol_block_select_pooled(const float* qbar, const float* kbar, sol_sha
 sol_status sol_sparse_attn_fwd(const void* q, const void* k, const void* v, const int32_t* idx,
                                sol_shape s, int block, int topk, float softmax_scale,
                                sol_dtype dt, void* o, float* lse, cudaStream_t stream);
+
+/*
+ * sol_sparse_attn_fwd_counts -- sol_sparse_attn_fwd where row (b,h,i) attends
+ * to the key blocks idx[b,h,i,0 .. c-1] only, c = counts[b,h,i] clamped to
+ * [1, topk] (the variable-length rows of sol_block_select_pooled_ex).
+ *
+ * counts : device int32 [B, H, nb], required (NULL: SOL_ERR_INVALID_ARG).
+ * idx keeps its row stride topk; entries at and beyond c are not read.
+ * Everything else as sol_sparse_attn_fwd; counts all equal to topk give its result.
+ */
+sol_status sol_sparse_attn_fwd_counts(const void* q, const void* k, const void* v, const int32_t* idx,
+                                      const int32_t* counts, sol_shape s, int block, int topk,
+                                      float softmax_scale, sol_dtype dt, void* o, float* lse,
+                                      cudaStream_t stream);
 
 /*
  * sol_block_select_noalloc -- sol_block_select for callers that cannot

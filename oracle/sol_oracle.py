@@ -42,7 +42,7 @@ import numpy as np
 __all__ = [
     "bf16_round", "rope_angles", "qk_prologue", "block_pool", "block_scores",
     "topk_blocks", "near_tie_rows", "block_select", "sparse_attention",
-    "sparse_attention_rows", "selected_flops",
+    "sparse_attention_rows", "selected_flops", "first_frame_blocks", "select_variant",
 ]
 
 
@@ -161,16 +161,69 @@ def block_select(q, k, block: int, topk: int):
     return topk_blocks(s, topk), s
 
 
-def sparse_attention_rows(q, k, v, idx, block: int, scale: float, b: int, h: int, i: int):
+def first_frame_blocks(grid, block: int) -> int:
+    """Number of blocks holding a token of frame t = 0: tokens 0 .. grid_h * grid_w - 1
+    come first in raster order, so blocks 0 .. ceil(grid_h * grid_w / block) - 1."""
+    return -(-(int(grid[1]) * int(grid[2])) // block)
+
+
+def select_variant(scores, topk: int, *, diagonal: bool = False, first_blocks: int = 0, top_p=None,
+                   scale: float = 1.0, head_k=None):
+    """Selection variants over a score matrix [B, H, nb, nb]: forced blocks, top-p, per-head k.
+
+    Sol-Attn decides per query which parts of the attention matter (ai-feiten.nl,
+    "Videomodel MiniMax-H3 rendert sneller dan afspelen", section "Waar de
+    snelheidswinst vandaan komt"); the pages fix no rule, so these are readings:
+      - forced blocks: the query's own block i (diagonal) and blocks 0 ..
+        first_blocks - 1 (the first latent frame) come first in the row's order,
+        in ascending id; the other blocks follow by descending score, exact ties
+        to the lower id;
+      - k_h = topk, or head_k[h] clamped to [1, topk];
+      - without top_p the row keeps the first k_h ids of its order; with top_p it
+        keeps the first c = min(k_h, max(#forced, 1, c_p)), where c_p is the
+        shortest prefix whose softmax mass, softmax_j(scale * s_ij) over all
+        key blocks, reaches top_p.
+    Returns (idx int32 [B, H, nb, topk]: the kept ids ascending, then -1;
+    counts int32 [B, H, nb]).
+    """
+    s = np.asarray(scores, np.float64)
+    B, H, nb, _ = s.shape
+    idx = np.full((B, H, nb, topk), -1, dtype=np.int32)
+    counts = np.zeros((B, H, nb), dtype=np.int32)
+    for b in range(B):
+        for h in range(H):
+            kh = topk if head_k is None else min(max(int(head_k[h]), 1), topk)
+            for i in range(nb):
+                row = s[b, h, i]
+                forced = set(range(min(first_blocks, nb)))
+                if diagonal:
+                    forced.add(i)
+                rest = [j for j in np.argsort(-row, kind="stable") if j not in forced]
+                order = sorted(forced) + rest
+                if top_p is None:
+                    c = kh
+                else:
+                    e = np.exp(scale * (row - row.max()))
+                    cum = np.cumsum(e[order])
+                    c_p = int(np.argmax(cum >= top_p * cum[-1])) + 1   # cum[-1]: the row's total mass
+                    c = min(kh, max(len(forced), 1, c_p))
+                idx[b, h, i, :c] = np.sort(np.asarray(order[:c]))
+                counts[b, h, i] = c
+    return idx, counts
+
+
+def sparse_attention_rows(q, k, v, idx, block: int, scale: float, b: int, h: int, i: int, count=None):
     """Attention of the queries of block i of (b, h) over its kept key blocks.
 
-    Keys: every token m < N of the blocks idx[b, h, i, :].  Logits
+    Keys: every token m < N of the blocks idx[b, h, i, :count] (all of the row
+    when count is None).  Logits
     l_m = scale * q_n . k_m; two-pass softmax: subtract the row max, exponentiate,
     normalise.  Returns (o [n_i, D], lse [n_i]) with lse = ln sum_m exp(l_m).
     """
     N = q.shape[1]
     rows = np.arange(i * block, min(N, (i + 1) * block))
-    cols = np.concatenate([np.arange(j * block, min(N, (j + 1) * block)) for j in np.asarray(idx[b, h, i])])
+    kept = np.asarray(idx[b, h, i])[:count]
+    cols = np.concatenate([np.arange(j * block, min(N, (j + 1) * block)) for j in kept])
     qi = np.asarray(q[b, rows, h, :], np.float64)
     kj = np.asarray(k[b, cols, h, :], np.float64)
     vj = np.asarray(v[b, cols, h, :], np.float64)
@@ -183,11 +236,12 @@ def sparse_attention_rows(q, k, v, idx, block: int, scale: float, b: int, h: int
     return o, lse
 
 
-def sparse_attention(q, k, v, idx, block: int, scale: float | None = None, units=None):
+def sparse_attention(q, k, v, idx, block: int, scale: float | None = None, units=None, counts=None):
     """Step a5 over all (b, h, query block) units, or over the listed `units`.
 
     q, k, v: [B, N, H, D] stored tensors (widened exactly to float64).
-    idx: [B, H, nb, k] kept key-block ids.  scale defaults to 1/sqrt(D).
+    idx: [B, H, nb, k] kept key-block ids; with counts [B, H, nb], row (b, h, i)
+    keeps only its first counts[b, h, i] ids.  scale defaults to 1/sqrt(D).
     Returns (o [B, N, H, D], lse [B, H, N]) float64; rows of units not computed
     are NaN.
     """
@@ -203,7 +257,8 @@ def sparse_attention(q, k, v, idx, block: int, scale: float | None = None, units
     if units is None:
         units = [(b, h, i) for b in range(B) for h in range(H) for i in range(nb)]
     for (b, h, i) in units:
-        oi, li = sparse_attention_rows(q, k, v, idx, block, scale, b, h, i)
+        c = None if counts is None else int(counts[b, h, i])
+        oi, li = sparse_attention_rows(q, k, v, idx, block, scale, b, h, i, c)
         r0, r1 = i * block, min(N, (i + 1) * block)
         o[b, r0:r1, h, :] = oi
         lse[b, h, r0:r1] = li

@@ -148,3 +148,43 @@ def test_select_pooled_argument_checks(lib):
     assert f(FAKE, FAKE, Shape(1, 1000, 2, 64, 4, 16, 16), 64, 4, FAKE, None, None) == INVALID
     big = Shape(1, 2049 * 64, 2, 64, 1, 2049, 64)                                 # nb = 2049 > 2048
     assert f(FAKE, FAKE, big, 64, 4, FAKE, None, None) == UNSUPPORTED
+
+
+class SelectOpts(ctypes.Structure):
+    _fields_ = [("flags", ctypes.c_uint), ("top_p", ctypes.c_float), ("softmax_scale", ctypes.c_float),
+                ("head_k", ctypes.c_void_p)]
+
+
+def test_select_pooled_ex_argument_checks(lib):
+    f = lib.sol_block_select_pooled_ex
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p, ctypes.c_void_p, Shape, ctypes.c_int, ctypes.c_int,
+                  ctypes.POINTER(SelectOpts), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+
+    def call(opts=SelectOpts(0, 1.0, 0.0, None), k=4, counts=FAKE, shape=OK_SHAPE, idx=FAKE):
+        return f(FAKE, FAKE, shape, 64, k, ctypes.byref(opts) if opts is not None else None, idx, counts, None, None)
+
+    assert call(opts=None) == INVALID
+    assert call(counts=None) == INVALID                                  # counts are required
+    assert call(counts=MISALIGNED) == INVALID
+    assert call(idx=None) == INVALID
+    assert call(k=0) == INVALID
+    assert call(k=17) == INVALID
+    assert call(opts=SelectOpts(8, 1.0, 0.0, None)) == INVALID            # unknown flag
+    assert call(opts=SelectOpts(4, 0.0, 0.0, None)) == INVALID            # top_p must be in (0, 1]
+    assert call(opts=SelectOpts(4, 1.5, 0.0, None)) == INVALID
+    assert call(opts=SelectOpts(4, float("nan"), 0.0, None)) == INVALID
+    assert call(opts=SelectOpts(4, 0.5, float("inf"), None)) == INVALID
+    big = Shape(1, 2049 * 64, 2, 64, 1, 2049, 64)
+    assert call(shape=big) == UNSUPPORTED
+
+
+def test_attention_counts_argument_checks(lib):
+    f = lib.sol_sparse_attn_fwd_counts
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p] * 5 + [Shape, ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_int,
+                                          ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+    assert f(FAKE, FAKE, FAKE, FAKE, None, OK_SHAPE, 64, 4, 0.0, 0, FAKE, FAKE, None) == INVALID   # no counts
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, OK_SHAPE, 64, 0, 0.0, 0, FAKE, FAKE, None) == INVALID
+    assert f(FAKE, FAKE, None, FAKE, FAKE, OK_SHAPE, 64, 4, 0.0, 0, FAKE, FAKE, None) == INVALID
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, OK_SHAPE, 64, 4, float("nan"), 0, FAKE, FAKE, None) == INVALID

@@ -13,6 +13,7 @@ import pytest
 import oracle
 import oracle.sol_oracle as so
 from tests import test_oracle_pins as pins
+from tests import test_oracle_variants as vpins
 
 
 def _prologue_rope_sign(x, gamma, grid, split, theta, eps):
@@ -69,18 +70,30 @@ def _topk_ties_high(scores, k):
     return np.sort(n - 1 - order, axis=-1).astype(np.int32)
 
 
-def _attention_rows_no_scale(q, k, v, idx, block, scale, b, h, i):
-    return so.__dict__["_orig_rows"](q, k, v, idx, block, 1.0, b, h, i)
+def _attention_rows_no_scale(q, k, v, idx, block, scale, b, h, i, count=None):
+    return so.__dict__["_orig_rows"](q, k, v, idx, block, 1.0, b, h, i, count)
 
 
-def _attention_rows_lse_no_max(q, k, v, idx, block, scale, b, h, i):
-    o, lse = so.__dict__["_orig_rows"](q, k, v, idx, block, scale, b, h, i)
+def _attention_rows_lse_no_max(q, k, v, idx, block, scale, b, h, i, count=None):
+    o, lse = so.__dict__["_orig_rows"](q, k, v, idx, block, scale, b, h, i, count)
     N = q.shape[1]
     rows = np.arange(i * block, min(N, (i + 1) * block))
-    cols = np.concatenate([np.arange(j * block, min(N, (j + 1) * block)) for j in np.asarray(idx[b, h, i])])
+    cols = np.concatenate([np.arange(j * block, min(N, (j + 1) * block)) for j in np.asarray(idx[b, h, i])[:count]])
     logits = scale * (np.asarray(q[b, rows, h], np.float64) @ np.asarray(k[b, cols, h], np.float64).T)
     mx = logits.max(axis=1)
     return o, lse - mx
+
+
+def _variant_diagonal_dropped(scores, topk, **kw):
+    return so.__dict__["_orig_variant"](scores, topk, **{**kw, "diagonal": False})
+
+
+def _variant_scale_ignored(scores, topk, **kw):
+    return so.__dict__["_orig_variant"](scores, topk, **{**kw, "scale": 1.0})
+
+
+def _variant_head_k_ignored(scores, topk, **kw):
+    return so.__dict__["_orig_variant"](scores, topk, **{**kw, "head_k": None})
 
 
 MUTATIONS = [
@@ -92,12 +105,16 @@ MUTATIONS = [
     ("sparse_attention_rows", _attention_rows_no_scale, [pins.test_attention_all_blocks_equals_dense_library_attention]),
     ("sparse_attention_rows", _attention_rows_lse_no_max, [pins.test_attention_all_blocks_equals_dense_library_attention,
                                                            pins.test_attention_hand_cases]),
+    ("select_variant", _variant_diagonal_dropped, [lambda: vpins.test_forced_diagonal_brute_force(2)]),
+    ("select_variant", _variant_scale_ignored, [lambda: vpins.test_top_p_count_is_smallest_subset_reaching_p(0.6)]),
+    ("select_variant", _variant_head_k_ignored, [vpins.test_per_head_k]),
 ]
 
 
 @pytest.mark.parametrize("name,bad,tests", MUTATIONS, ids=[m[1].__name__ for m in MUTATIONS])
 def test_pins_catch_planted_mistake(monkeypatch, name, bad, tests):
     monkeypatch.setitem(so.__dict__, "_orig_rows", so.sparse_attention_rows)
+    monkeypatch.setitem(so.__dict__, "_orig_variant", so.select_variant)
     monkeypatch.setattr(so, name, bad)
     monkeypatch.setattr(oracle, name, bad)
     for t in tests:
