@@ -52,7 +52,8 @@ def load_peaks():
 
 
 KERNEL_SOURCES = ("block_sparse_attention_sol_b200/csrc/attn_sm100.cuh",
-                  "block_sparse_attention_sol_b200/csrc/sm100_ptx.cuh")
+                  "block_sparse_attention_sol_b200/csrc/sm100_ptx.cuh",
+                  "block_sparse_attention_sol_b200/csrc/blocks.cuh")
 
 
 def load_ncu_traffic(kernel: str):

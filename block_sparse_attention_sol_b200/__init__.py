@@ -13,6 +13,8 @@ Functions (same names as the C ABI):
     sol_block_select_pooled(qbar, kbar, grid, block, topk, ...) -> idx [, scores]
     sol_block_select_pooled_ex(qbar, kbar, grid, block, topk, flags=..., ...) -> (idx, counts) [, scores]
     sol_sparse_attn_fwd_counts(q, k, v, idx, counts, grid, block, ...) -> (o, lse)
+    sol_qk_prologue_pool_tiled(q_raw, k_raw, gamma_q, gamma_k, grid, tile, ...) -> (q, k, qbar, kbar)
+    sol_sparse_attn_fwd_tiled(q, k, v, idx, grid, tile, counts=None, ...) -> (o, lse)
     sol_check_device_status(stream=None)
     sol_selftest_wait_timeout(limit_us, stream=None)
     sol_block_select_workspace_bytes(shape, block)
@@ -28,7 +30,7 @@ __all__ = [
     "SolError", "SolShape", "LIB_PATH", "lib",
     "sol_qk_prologue", "sol_block_select", "sol_block_select_workspace_bytes", "sol_sparse_attn_fwd",
     "sol_qk_prologue_pool", "sol_block_select_pooled", "sol_block_select_pooled_ex", "sol_sparse_attn_fwd_counts",
-    "SolSelectOpts", "SOL_SELECT_FORCE_DIAGONAL", "SOL_SELECT_FORCE_FIRST_FRAME", "SOL_SELECT_TOP_P",
+    "SolSelectOpts", "SolTile", "sol_qk_prologue_pool_tiled", "sol_sparse_attn_fwd_tiled", "SOL_SELECT_FORCE_DIAGONAL", "SOL_SELECT_FORCE_FIRST_FRAME", "SOL_SELECT_TOP_P",
     "sol_check_device_status", "sol_selftest_wait_timeout", "sol_status_string", "sol_attention_chain",
     "SOL_OK", "SOL_ERR_INVALID_ARG", "SOL_ERR_UNSUPPORTED", "SOL_ERR_CUDA", "SOL_ERR_TIMEOUT",
 ]
@@ -49,9 +51,13 @@ class SolShape(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in ("B", "N", "H", "D", "grid_t", "grid_h", "grid_w")]
 
 
+class SolTile(ctypes.Structure):
+    _fields_ = [("t", ctypes.c_int), ("h", ctypes.c_int), ("w", ctypes.c_int)]
+
+
 class SolSelectOpts(ctypes.Structure):
     _fields_ = [("flags", ctypes.c_uint), ("top_p", ctypes.c_float), ("softmax_scale", ctypes.c_float),
-                ("head_k", ctypes.c_void_p)]
+                ("head_k", ctypes.c_void_p), ("tile", SolTile)]
 
 
 class SolError(RuntimeError):
@@ -77,6 +83,11 @@ lib.sol_block_select_pooled_ex.restype = _I
 lib.sol_block_select_pooled_ex.argtypes = [_P, _P, SolShape, _I, _I, ctypes.POINTER(SolSelectOpts), _P, _P, _P, _P]
 lib.sol_sparse_attn_fwd_counts.restype = _I
 lib.sol_sparse_attn_fwd_counts.argtypes = [_P, _P, _P, _P, _P, SolShape, _I, _I, _F, _I, _P, _P, _P]
+lib.sol_qk_prologue_pool_tiled.restype = _I
+lib.sol_qk_prologue_pool_tiled.argtypes = [_P, _P, _P, _P, _P, _P, SolShape, _I, _I, _I, _F, _F, _I, SolTile, _P, _P,
+                                           _P]
+lib.sol_sparse_attn_fwd_tiled.restype = _I
+lib.sol_sparse_attn_fwd_tiled.argtypes = [_P, _P, _P, _P, _P, SolShape, SolTile, _I, _F, _I, _P, _P, _P]
 lib.sol_sparse_attn_fwd.restype = _I
 lib.sol_sparse_attn_fwd.argtypes = [_P, _P, _P, _P, SolShape, _I, _I, _F, _I, _P, _P, _P]
 lib.sol_check_device_status.restype = _I
@@ -165,6 +176,33 @@ def sol_qk_prologue_pool(q_raw, k_raw, gamma_q, gamma_k, grid, block, rope_split
     return q_out, k_out, qbar_out, kbar_out
 
 
+def sol_qk_prologue_pool_tiled(q_raw, k_raw, gamma_q, gamma_k, grid, tile, rope_split=None, rope_theta=10000.0,
+                               eps=1e-6, q_out=None, k_out=None, qbar_out=None, kbar_out=None, stream=None):
+    """sol_qk_prologue plus the fp32 means of its stored outputs over 3-D tiles
+    tile = (t, h, w).  Returns (q, k, qbar, kbar); qbar, kbar are [B, H, N / (t h w), D]."""
+    _cuda(q_raw, "q_raw"), _cuda(k_raw, "k_raw"), _cuda(gamma_q, "gamma_q"), _cuda(gamma_k, "gamma_k")
+    s = _shape(q_raw, grid)
+    if rope_split is None:
+        dh = 2 * (s.D // 6)
+        rope_split = (s.D - 2 * dh, dh, dh)
+    block = int(tile[0]) * int(tile[1]) * int(tile[2])
+    nb = max(s.N // block, 1)
+    q_out = torch.empty_like(q_raw) if q_out is None else _cuda(q_out, "q_out")
+    k_out = torch.empty_like(k_raw) if k_out is None else _cuda(k_out, "k_out")
+    pooled = (s.B, s.H, nb, s.D)
+    qbar_out = (torch.empty(pooled, dtype=torch.float32, device=q_raw.device) if qbar_out is None
+                else _cuda(qbar_out, "qbar_out"))
+    kbar_out = (torch.empty(pooled, dtype=torch.float32, device=q_raw.device) if kbar_out is None
+                else _cuda(kbar_out, "kbar_out"))
+    st = lib.sol_qk_prologue_pool_tiled(q_raw.data_ptr(), k_raw.data_ptr(), q_out.data_ptr(), k_out.data_ptr(),
+                                        gamma_q.data_ptr(), gamma_k.data_ptr(), s, int(rope_split[0]),
+                                        int(rope_split[1]), int(rope_split[2]), float(rope_theta), float(eps),
+                                        _dtype_code(q_raw), SolTile(*(int(x) for x in tile)), qbar_out.data_ptr(),
+                                        kbar_out.data_ptr(), _stream_handle(stream))
+    _check(st, "sol_qk_prologue_pool_tiled")
+    return q_out, k_out, qbar_out, kbar_out
+
+
 def sol_block_select_pooled(qbar, kbar, grid, block, topk, idx_out=None, return_scores=False, stream=None):
     """Scores + top-k from block means [B, H, nb, D] (fp32).  Returns idx (and the scores)."""
     _cuda(qbar, "qbar"), _cuda(kbar, "kbar")
@@ -184,7 +222,7 @@ def sol_block_select_pooled(qbar, kbar, grid, block, topk, idx_out=None, return_
 
 
 def sol_block_select_pooled_ex(qbar, kbar, grid, block, topk, flags=0, top_p=1.0, softmax_scale=0.0, head_k=None,
-                               idx_out=None, counts_out=None, return_scores=False, stream=None):
+                               tile=None, idx_out=None, counts_out=None, return_scores=False, stream=None):
     """Selection variants (forced diagonal / first-frame blocks, top-p, per-head k)
     from block means.  Returns (idx, counts) (and the scores); rows of idx hold
     their count of ascending ids, then -1."""
@@ -204,7 +242,8 @@ def sol_block_select_pooled_ex(qbar, kbar, grid, block, topk, flags=0, top_p=1.0
         counts_out = torch.empty((B, H, nb), dtype=torch.int32, device=qbar.device)
     scores = torch.empty((B, H, nb, nb), dtype=torch.float32, device=qbar.device) if return_scores else None
     opts = SolSelectOpts(int(flags), float(top_p), float(softmax_scale),
-                         head_k.data_ptr() if head_k is not None else None)
+                         head_k.data_ptr() if head_k is not None else None,
+                         SolTile(*(int(x) for x in tile)) if tile is not None else SolTile(0, 0, 0))
     st = lib.sol_block_select_pooled_ex(qbar.data_ptr(), kbar.data_ptr(), s, int(block), int(topk),
                                         ctypes.byref(opts), _cuda(idx_out, "idx_out").data_ptr(),
                                         _cuda(counts_out, "counts_out").data_ptr(),
@@ -267,6 +306,24 @@ def sol_sparse_attn_fwd_counts(q, k, v, idx, counts, grid, block, softmax_scale=
                                         s, int(block), int(topk), float(softmax_scale), _dtype_code(q), o.data_ptr(),
                                         lse.data_ptr(), _stream_handle(stream))
     _check(st, "sol_sparse_attn_fwd_counts")
+    return o, lse
+
+
+def sol_sparse_attn_fwd_tiled(q, k, v, idx, grid, tile, counts=None, softmax_scale=0.0, o=None, lse=None,
+                              stream=None):
+    """Attention over 3-D tile blocks tile = (t, h, w) (optionally count-limited rows).  Returns (o, lse)."""
+    _cuda(q, "q"), _cuda(k, "k"), _cuda(v, "v"), _cuda(idx, "idx")
+    if idx.dtype != torch.int32 or (counts is not None and counts.dtype != torch.int32):
+        raise TypeError("idx and counts must be int32")
+    s = _shape(q, grid)
+    topk = idx.shape[-1]
+    o = torch.empty_like(q) if o is None else _cuda(o, "o")
+    lse = torch.empty((s.B, s.H, s.N), dtype=torch.float32, device=q.device) if lse is None else _cuda(lse, "lse")
+    st = lib.sol_sparse_attn_fwd_tiled(q.data_ptr(), k.data_ptr(), v.data_ptr(), idx.data_ptr(),
+                                       _cuda(counts, "counts").data_ptr() if counts is not None else None, s,
+                                       SolTile(*(int(x) for x in tile)), int(topk), float(softmax_scale),
+                                       _dtype_code(q), o.data_ptr(), lse.data_ptr(), _stream_handle(stream))
+    _check(st, "sol_sparse_attn_fwd_tiled")
     return o, lse
 
 

@@ -8,6 +8,7 @@
 // shuffles.  Online softmax with exact expf, fp32 throughout.
 #pragma once
 #include <cstdint>
+#include "blocks.cuh"
 
 namespace sol {
 namespace attnf32 {
@@ -18,7 +19,7 @@ template <int D>
 __global__ void __launch_bounds__(kWarps * 32) sparse_attn_fwd_f32_kernel(
     const float* __restrict__ q, const float* __restrict__ k, const float* __restrict__ v,
     const int32_t* __restrict__ idx, const int32_t* __restrict__ counts, float* __restrict__ o,
-    float* __restrict__ lse, int B, int N, int H, int block, int nb, int topk, float scale) {
+    float* __restrict__ lse, int B, int N, int H, const BlockMap bm, int nb, int topk, float scale) {
   constexpr int C = D / 32;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long row = static_cast<long long>(blockIdx.x) * kWarps + warp;   // over B * H * N
@@ -31,14 +32,15 @@ __global__ void __launch_bounds__(kWarps * 32) sparse_attn_fwd_f32_kernel(
   float qr[C], acc[C];
 #pragma unroll
   for (int c = 0; c < C; ++c) { qr[c] = qp[lane + 32 * c] * scale; acc[c] = 0.f; }
-  const size_t rowi = static_cast<size_t>(b * H + h) * nb + n / block;   // row of idx / counts
+  const size_t rowi = static_cast<size_t>(b * H + h) * nb + token_block(bm, n);   // row of idx / counts
   const int32_t* list = idx + rowi * topk;
   const int kt = counts == nullptr ? topk : min(max(counts[rowi], 1), topk);
   float m = -INFINITY, l = 0.f;
   for (int j = 0; j < kt; ++j) {
     const int blk = list[j];
-    const int m0 = blk * block, m1 = min(N, m0 + block);
-    for (int mk = m0; mk < m1; ++mk) {
+    const int len = bm.tw == 0 ? min(bm.block, N - blk * bm.block) : bm.block;
+    for (int u = 0; u < len; ++u) {
+      const int mk = block_token(bm, blk, u);
       const float* kp = k + (static_cast<size_t>(b) * N + mk) * rs + h * D;
       float part = 0.f;
 #pragma unroll

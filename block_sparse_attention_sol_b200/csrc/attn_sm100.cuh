@@ -35,6 +35,7 @@
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include "blocks.cuh"
 #include "sm100_ptx.cuh"
 
 namespace sol {
@@ -75,6 +76,8 @@ struct Params {
   int B, N, H, nb, topk;
   int num_tiles;
   float scale_log2;       // softmax scale * log2(e)
+  BlockMap bm;            // token blocks (block == kBlock); tiled: K/V maps are 5-D (c, h, x, y, b * T + t)
+  int T;                  // frames of the grid
 };
 
 // Wait-site ids reported in the error info word.
@@ -90,6 +93,22 @@ __device__ __forceinline__ constexpr uint32_t kstep_off(int kk) {
 // Key blocks of tile t (row t of idx in [B, H, nb] order); every role reads the same value.
 __device__ __forceinline__ int tile_steps(const Params& p, int t) {
   return p.counts == nullptr ? p.topk : min(max(__ldg(p.counts + t), 1), p.topk);
+}
+
+// Both 64-channel halves of key block `blk` of (b, h) into a slot: one 4-D box of
+// 128 consecutive tokens, or one 5-D box of a tt x th x tw tile (rows in the
+// same tile-raster order as block_token).
+__device__ __forceinline__ void load_block(uint8_t* dst, const CUtensorMap* tm, uint64_t* bar, const Params& p, int blk,
+                                           int h, int b) {
+  if (p.bm.tw == 0) {
+    tma_load_4d(dst, tm, bar, 0, h, blk * kBlock, b);
+    tma_load_4d(dst + kHalfBytes, tm, bar, 64, h, blk * kBlock, b);
+  } else {
+    int t0, y0, x0;
+    tile_origin(p.bm, blk, t0, y0, x0);
+    tma_load_5d(dst, tm, bar, 0, h, x0, y0, b * p.T + t0);
+    tma_load_5d(dst + kHalfBytes, tm, bar, 64, h, x0, y0, b * p.T + t0);
+  }
 }
 
 __device__ __forceinline__ void decode_tile(const Params& p, int t, int& b, int& h, int& qb) {
@@ -146,16 +165,8 @@ sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
           if (use > 0 && !(ok = mbar_wait(&sm.slot_done[st], (use - 1) & 1, abort_flag, kSiteSlotFree))) break;
           const bool has_k = s < kt, has_v = s >= 2;
           mbar_arrive_expect_tx(&sm.kv_full[st], (has_k ? kTileBytes : 0) + (has_v ? kTileBytes : 0));
-          if (has_k) {
-            const int blk = __ldg(list + s);
-            tma_load_4d(sm.k[st], &tm_k, &sm.kv_full[st], 0, h, blk * kBlock, b);
-            tma_load_4d(sm.k[st] + kHalfBytes, &tm_k, &sm.kv_full[st], 64, h, blk * kBlock, b);
-          }
-          if (has_v) {
-            const int blk = __ldg(list + s - 2);
-            tma_load_4d(sm.v[st], &tm_v, &sm.kv_full[st], 0, h, blk * kBlock, b);
-            tma_load_4d(sm.v[st] + kHalfBytes, &tm_v, &sm.kv_full[st], 64, h, blk * kBlock, b);
-          }
+          if (has_k) load_block(sm.k[st], &tm_k, &sm.kv_full[st], p, __ldg(list + s), h, b);
+          if (has_v) load_block(sm.v[st], &tm_v, &sm.kv_full[st], p, __ldg(list + s - 2), h, b);
         }
       }
       // Before the CTA exits, every load issued must have landed (slot s was
@@ -261,7 +272,7 @@ sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
         tc_fence_after();
       }
       {
-        const int nq = qb * kBlock + quad * 32 + lane;
+        const int nq = block_token(p.bm, qb, quad * 32 + lane);
         uint32_t qv[32];
         if (nq < p.N) {
           const uint4* src = reinterpret_cast<const uint4*>(
@@ -420,10 +431,9 @@ sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.o_free);
-      const int n0 = qb * kBlock + row0;
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
-        const int n = n0 + 8 * u;
+        const int n = block_token(p.bm, qb, row0 + 8 * u);
         if (n < p.N) {
           uint32_t* dst = reinterpret_cast<uint32_t*>(p.o + ((static_cast<size_t>(b) * p.N + n) * p.H + h) * kHeadDim);
 #pragma unroll

@@ -20,6 +20,7 @@
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
+#include "blocks.cuh"
 
 namespace sol {
 namespace prologue {
@@ -205,9 +206,10 @@ __device__ __forceinline__ void store_vec_acc(__nv_bfloat16* p, const float (&y)
   *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-// grid (nb, B); qbar, kbar: fp32 [B, H, nb, D].
+// grid (nb, B); qbar, kbar: fp32 [B, H, nb, D].  Block bi holds the tokens
+// block_token(bm, bi, l), l = 0 .. its length - 1, summed in that order.
 template <typename T, int D>
-__global__ void __launch_bounds__(256) qk_prologue_pool_kernel(const Params p, int block, int nb, float* qbar,
+__global__ void __launch_bounds__(256) qk_prologue_pool_kernel(const Params p, const BlockMap bm, int nb, float* qbar,
                                                                float* kbar) {
   extern __shared__ float2 tab[];   // [gt * dt/2 | gh * dh/2 | gw * dw/2] of (cos, sin)
   const int pt = p.dt / 2, ph = p.dh / 2, pw = p.dw / 2;
@@ -231,9 +233,8 @@ __global__ void __launch_bounds__(256) qk_prologue_pool_kernel(const Params p, i
   const unsigned seg = (L == 32) ? 0xffffffffu : (((1u << (L & 31)) - 1u) << (lane & ~(unsigned)(L - 1)));
   const int grp = threadIdx.x / L;
   const int bi = blockIdx.x, b = blockIdx.y;
-  const int n0 = bi * block;
-  const int n1 = min(n0 + block, p.N);
-  const float inv = 1.0f / static_cast<float>(n1 - n0);
+  const int cnt = bm.tw == 0 ? min(bm.block, p.N - bi * bm.block) : bm.block;   // tokens of this block
+  const float inv = 1.0f / static_cast<float>(cnt);
 
   int axis[V / 2], slot[V / 2];
 #pragma unroll
@@ -266,9 +267,10 @@ __global__ void __launch_bounds__(256) qk_prologue_pool_kernel(const Params p, i
     }
     const size_t base = (static_cast<size_t>(b) * p.N * p.H + h) * D + lane_in_row * V;
     const size_t tstride = static_cast<size_t>(p.H) * D;
-    int n = n0;
-    for (; n + 1 < n1; n += 2) {   // two tokens in flight
-      const size_t o1 = base + static_cast<size_t>(n) * tstride, o2 = o1 + tstride;
+    int l = 0;
+    for (; l + 1 < cnt; l += 2) {   // two tokens in flight
+      const int n = block_token(bm, bi, l), n2 = block_token(bm, bi, l + 1);
+      const size_t o1 = base + static_cast<size_t>(n) * tstride, o2 = base + static_cast<size_t>(n2) * tstride;
       float xq1[V], xk1[V], xq2[V], xk2[V];
       load_vec(qi + o1, xq1);
       load_vec(ki + o1, xk1);
@@ -276,7 +278,7 @@ __global__ void __launch_bounds__(256) qk_prologue_pool_kernel(const Params p, i
       load_vec(ki + o2, xk2);
       float2 cs1[V / 2], cs2[V / 2];
       angles(n, cs1);
-      angles(n + 1, cs2);
+      angles(n2, cs2);
       norm_rotate<V, L>(xq1, gq, cs1, seg, D, p.eps);
       norm_rotate<V, L>(xk1, gk, cs1, seg, D, p.eps);
       norm_rotate<V, L>(xq2, gq, cs2, seg, D, p.eps);
@@ -286,7 +288,8 @@ __global__ void __launch_bounds__(256) qk_prologue_pool_kernel(const Params p, i
       store_vec_acc(qo + o2, xq2, aq);
       store_vec_acc(ko + o2, xk2, ak);
     }
-    if (n < n1) {
+    if (l < cnt) {
+      const int n = block_token(bm, bi, l);
       const size_t o1 = base + static_cast<size_t>(n) * tstride;
       float xq[V], xk[V];
       load_vec(qi + o1, xq);

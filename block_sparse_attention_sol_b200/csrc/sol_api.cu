@@ -18,6 +18,7 @@
 #include "../../include/sol.h"
 #include "sm100_ptx.cuh"
 #include "attn_f32.cuh"
+#include "blocks.cuh"
 #include "attn_sm100.cuh"
 #include "prologue.cuh"
 #include "select.cuh"
@@ -96,6 +97,39 @@ sol_status make_bshd_map(CUtensorMap* map, const void* base, const sol_shape& s)
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? SOL_OK : SOL_ERR_CUDA;
+}
+
+// 5-D view (channel, head, x, y, b * T + t) of a [B, N, H, D] bf16 tensor whose
+// tokens are the grid in raster order; a box is 64 channels of one head over a
+// tw x th x tt tile of tokens, rows in tile-raster order (x fastest).
+sol_status make_tile_map(CUtensorMap* map, const void* base, const sol_shape& s, const sol::BlockMap& bm) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return SOL_ERR_CUDA;
+  const cuuint64_t row = static_cast<cuuint64_t>(s.H) * s.D * 2;   // bytes per token
+  cuuint64_t dims[5] = {static_cast<cuuint64_t>(s.D), static_cast<cuuint64_t>(s.H),
+                        static_cast<cuuint64_t>(s.grid_w), static_cast<cuuint64_t>(s.grid_h),
+                        static_cast<cuuint64_t>(s.grid_t) * s.B};
+  cuuint64_t strides[4] = {static_cast<cuuint64_t>(s.D) * 2, row, row * s.grid_w, row * s.grid_w * s.grid_h};
+  cuuint32_t box[5] = {64, 1, static_cast<cuuint32_t>(bm.tw), static_cast<cuuint32_t>(bm.th),
+                       static_cast<cuuint32_t>(bm.tt)};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? SOL_OK : SOL_ERR_CUDA;
+}
+
+// Block map of 3-D tiles that cover the grid exactly, or SOL_ERR_INVALID_ARG.
+sol_status tile_blocks(const sol_shape& s, sol_tile tile, sol::BlockMap* out) {
+  if (tile.t < 1 || tile.h < 1 || tile.w < 1) return SOL_ERR_INVALID_ARG;
+  if (s.grid_t % tile.t || s.grid_h % tile.h || s.grid_w % tile.w) return SOL_ERR_INVALID_ARG;
+  if (static_cast<long long>(tile.t) * tile.h * tile.w > 4096) return SOL_ERR_UNSUPPORTED;
+  *out = sol::tiled_blocks(tile.t, tile.h, tile.w, s.grid_h, s.grid_w);
+  return SOL_OK;
+}
+
+int blocks_of(const sol_shape& s, const sol::BlockMap& bm) {
+  return bm.tw == 0 ? num_blocks(s.N, bm.block) : s.N / bm.block;
 }
 
 sol_status launch_status() { return cudaGetLastError() == cudaSuccess ? SOL_OK : SOL_ERR_CUDA; }
@@ -221,13 +255,44 @@ sol_status prologue_params(const void* q_raw, const void* k_raw, void* q_out, vo
   return SOL_OK;
 }
 
+// The fused prologue + block means for any block map.
+sol_status prologue_pool_impl(const void* q_raw, const void* k_raw, void* q_out, void* k_out, const float* gamma_q,
+                              const float* gamma_k, sol_shape s, int rope_dt, int rope_dh, int rope_dw,
+                              float rope_theta, float eps, sol_dtype dt, const sol::BlockMap& bm, float* qbar_out,
+                              float* kbar_out, cudaStream_t stream) {
+  sol::prologue::Params p;
+  size_t smem = 0;
+  if (sol_status st = prologue_params(q_raw, k_raw, q_out, k_out, gamma_q, gamma_k, s, rope_dt, rope_dh, rope_dw,
+                                      rope_theta, eps, dt, &p, &smem))
+    return st;
+  if (!qbar_out || !kbar_out || !aligned16(qbar_out) || !aligned16(kbar_out) || bm.block <= 0)
+    return SOL_ERR_INVALID_ARG;
+  const int nb = blocks_of(s, bm);
+  if (nb > 65535 || s.B > 65535) return SOL_ERR_UNSUPPORTED;
+  const dim3 grid(nb, s.B);
+  if (dt == SOL_BF16) {
+    if (s.D == 128)
+      sol::prologue::qk_prologue_pool_kernel<__nv_bfloat16, 128><<<grid, 256, smem, stream>>>(p, bm, nb, qbar_out,
+                                                                                              kbar_out);
+    else
+      sol::prologue::qk_prologue_pool_kernel<__nv_bfloat16, 64><<<grid, 256, smem, stream>>>(p, bm, nb, qbar_out,
+                                                                                             kbar_out);
+  } else {
+    if (s.D == 128)
+      sol::prologue::qk_prologue_pool_kernel<float, 128><<<grid, 256, smem, stream>>>(p, bm, nb, qbar_out, kbar_out);
+    else
+      sol::prologue::qk_prologue_pool_kernel<float, 64><<<grid, 256, smem, stream>>>(p, bm, nb, qbar_out, kbar_out);
+  }
+  return launch_status();
+}
+
 }  // namespace
 
 namespace {
 // Attention with optional per-row block counts (both attention entry points).
 sol_status sparse_attn_impl(const void* q, const void* k, const void* v, const int32_t* idx, const int32_t* counts,
-                            sol_shape s, int block, int topk, float softmax_scale, sol_dtype dt, void* o, float* lse,
-                            cudaStream_t stream);
+                            sol_shape s, const sol::BlockMap& bm, int topk, float softmax_scale, sol_dtype dt, void* o,
+                            float* lse, cudaStream_t stream);
 }  // namespace
 
 extern "C" {
@@ -280,30 +345,20 @@ sol_status sol_qk_prologue_pool(const void* q_raw, const void* k_raw, void* q_ou
                                 const float* gamma_k, sol_shape s, int rope_dt, int rope_dh, int rope_dw,
                                 float rope_theta, float eps, sol_dtype dt, int block, float* qbar_out,
                                 float* kbar_out, cudaStream_t stream) {
-  sol::prologue::Params p;
-  size_t smem = 0;
-  if (sol_status st = prologue_params(q_raw, k_raw, q_out, k_out, gamma_q, gamma_k, s, rope_dt, rope_dh, rope_dw,
-                                      rope_theta, eps, dt, &p, &smem))
-    return st;
-  if (!qbar_out || !kbar_out || !aligned16(qbar_out) || !aligned16(kbar_out) || block <= 0)
-    return SOL_ERR_INVALID_ARG;
-  const int nb = num_blocks(s.N, block);
-  if (nb > 65535 || s.B > 65535) return SOL_ERR_UNSUPPORTED;
-  const dim3 grid(nb, s.B);
-  if (dt == SOL_BF16) {
-    if (s.D == 128)
-      sol::prologue::qk_prologue_pool_kernel<__nv_bfloat16, 128><<<grid, 256, smem, stream>>>(p, block, nb, qbar_out,
-                                                                                              kbar_out);
-    else
-      sol::prologue::qk_prologue_pool_kernel<__nv_bfloat16, 64><<<grid, 256, smem, stream>>>(p, block, nb, qbar_out,
-                                                                                             kbar_out);
-  } else {
-    if (s.D == 128)
-      sol::prologue::qk_prologue_pool_kernel<float, 128><<<grid, 256, smem, stream>>>(p, block, nb, qbar_out, kbar_out);
-    else
-      sol::prologue::qk_prologue_pool_kernel<float, 64><<<grid, 256, smem, stream>>>(p, block, nb, qbar_out, kbar_out);
-  }
-  return launch_status();
+  if (block <= 0) return SOL_ERR_INVALID_ARG;
+  return prologue_pool_impl(q_raw, k_raw, q_out, k_out, gamma_q, gamma_k, s, rope_dt, rope_dh, rope_dw, rope_theta,
+                            eps, dt, sol::raster_blocks(block, s.grid_h, s.grid_w), qbar_out, kbar_out, stream);
+}
+
+sol_status sol_qk_prologue_pool_tiled(const void* q_raw, const void* k_raw, void* q_out, void* k_out,
+                                      const float* gamma_q, const float* gamma_k, sol_shape s, int rope_dt,
+                                      int rope_dh, int rope_dw, float rope_theta, float eps, sol_dtype dt,
+                                      sol_tile tile, float* qbar_out, float* kbar_out, cudaStream_t stream) {
+  if (!shape_ok(s)) return SOL_ERR_INVALID_ARG;
+  sol::BlockMap bm;
+  if (sol_status st = tile_blocks(s, tile, &bm)) return st;
+  return prologue_pool_impl(q_raw, k_raw, q_out, k_out, gamma_q, gamma_k, s, rope_dt, rope_dh, rope_dw, rope_theta,
+                            eps, dt, bm, qbar_out, kbar_out, stream);
 }
 
 size_t sol_block_select_workspace_bytes(sol_shape s, int block) {
@@ -372,6 +427,16 @@ sol_status sol_block_select_pooled_ex(const float* qbar, const float* kbar, sol_
   if (topp && !std::isfinite(opts->softmax_scale)) return SOL_ERR_INVALID_ARG;
   const int nb = num_blocks(s.N, block);
   if (topk < 1 || topk > nb) return SOL_ERR_INVALID_ARG;
+  // blocks holding a token of frame t = 0: tokens 0 .. grid_h * grid_w - 1 of runs of `block`
+  // tokens, or the tiles of the first tile layer
+  int n_first = num_blocks(s.grid_h * s.grid_w, block);
+  const sol_tile tile = opts->tile;
+  if (tile.t != 0 || tile.h != 0 || tile.w != 0) {
+    sol::BlockMap bm;
+    if (sol_status st = tile_blocks(s, tile, &bm)) return st;
+    if (bm.block != block) return SOL_ERR_INVALID_ARG;
+    n_first = bm.nty * bm.ntx;
+  }
   ScorePlan plan;
   if (sol_status st = plan_scores(s, nb, &plan)) return st;
   DeviceInfo* di = nullptr;
@@ -382,8 +447,7 @@ sol_status sol_block_select_pooled_ex(const float* qbar, const float* kbar, sol_
   a.flags = (opts->flags & SOL_SELECT_FORCE_DIAGONAL ? sol::select::kForceDiagonal : 0u) |
             (opts->flags & SOL_SELECT_FORCE_FIRST_FRAME ? sol::select::kForceFirstFrame : 0u) |
             (topp ? sol::select::kTopP : 0u);
-  // blocks holding a token of frame t = 0: tokens 0 .. grid_h * grid_w - 1 in raster order
-  a.n_first = num_blocks(s.grid_h * s.grid_w, block);
+  a.n_first = n_first;
   a.top_p = opts->top_p;
   const float scale = opts->softmax_scale > 0.f ? opts->softmax_scale : 1.0f / std::sqrt(static_cast<float>(s.D));
   a.scale_log2 = scale * 1.4426950408889634f;   // log2(e)
@@ -393,14 +457,26 @@ sol_status sol_block_select_pooled_ex(const float* qbar, const float* kbar, sol_
 sol_status sol_sparse_attn_fwd(const void* q, const void* k, const void* v, const int32_t* idx, sol_shape s,
                                int block, int topk, float softmax_scale, sol_dtype dt, void* o, float* lse,
                                cudaStream_t stream) {
-  return sparse_attn_impl(q, k, v, idx, nullptr, s, block, topk, softmax_scale, dt, o, lse, stream);
+  if (block <= 0) return SOL_ERR_INVALID_ARG;
+  return sparse_attn_impl(q, k, v, idx, nullptr, s, sol::raster_blocks(block, s.grid_h, s.grid_w), topk,
+                          softmax_scale, dt, o, lse, stream);
 }
 
 sol_status sol_sparse_attn_fwd_counts(const void* q, const void* k, const void* v, const int32_t* idx,
                                       const int32_t* counts, sol_shape s, int block, int topk, float softmax_scale,
                                       sol_dtype dt, void* o, float* lse, cudaStream_t stream) {
-  if (!counts) return SOL_ERR_INVALID_ARG;
-  return sparse_attn_impl(q, k, v, idx, counts, s, block, topk, softmax_scale, dt, o, lse, stream);
+  if (!counts || block <= 0) return SOL_ERR_INVALID_ARG;
+  return sparse_attn_impl(q, k, v, idx, counts, s, sol::raster_blocks(block, s.grid_h, s.grid_w), topk,
+                          softmax_scale, dt, o, lse, stream);
+}
+
+sol_status sol_sparse_attn_fwd_tiled(const void* q, const void* k, const void* v, const int32_t* idx,
+                                     const int32_t* counts, sol_shape s, sol_tile tile, int topk, float softmax_scale,
+                                     sol_dtype dt, void* o, float* lse, cudaStream_t stream) {
+  if (!shape_ok(s)) return SOL_ERR_INVALID_ARG;
+  sol::BlockMap bm;
+  if (sol_status st = tile_blocks(s, tile, &bm)) return st;
+  return sparse_attn_impl(q, k, v, idx, counts, s, bm, topk, softmax_scale, dt, o, lse, stream);
 }
 
 }  // extern "C"
@@ -408,14 +484,14 @@ sol_status sol_sparse_attn_fwd_counts(const void* q, const void* k, const void* 
 namespace {
 
 sol_status sparse_attn_impl(const void* q, const void* k, const void* v, const int32_t* idx, const int32_t* counts,
-                            sol_shape s, int block, int topk, float softmax_scale, sol_dtype dt, void* o, float* lse,
-                            cudaStream_t stream) {
+                            sol_shape s, const sol::BlockMap& bm, int topk, float softmax_scale, sol_dtype dt, void* o,
+                            float* lse, cudaStream_t stream) {
   if (!q || !k || !v || !idx || !o || !lse) return SOL_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(idx) || !aligned16(lse))
     return SOL_ERR_INVALID_ARG;
-  if (!shape_ok(s) || block <= 0) return SOL_ERR_INVALID_ARG;
+  if (!shape_ok(s) || bm.block <= 0) return SOL_ERR_INVALID_ARG;
   if (dt != SOL_F32 && dt != SOL_BF16) return SOL_ERR_INVALID_ARG;
-  const int nb = num_blocks(s.N, block);
+  const int nb = blocks_of(s, bm);
   if (topk < 1 || topk > nb) return SOL_ERR_INVALID_ARG;
   if (!std::isfinite(softmax_scale)) return SOL_ERR_INVALID_ARG;
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(s.D));
@@ -431,20 +507,20 @@ sol_status sparse_attn_impl(const void* q, const void* k, const void* v, const i
     if (s.D == 128)
       sol::attnf32::sparse_attn_fwd_f32_kernel<128><<<static_cast<int>(grid), sol::attnf32::kWarps * 32, 0, stream>>>(
           static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v), idx, counts,
-          static_cast<float*>(o), lse, s.B, s.N, s.H, block, nb, topk, scale);
+          static_cast<float*>(o), lse, s.B, s.N, s.H, bm, nb, topk, scale);
     else
       sol::attnf32::sparse_attn_fwd_f32_kernel<64><<<static_cast<int>(grid), sol::attnf32::kWarps * 32, 0, stream>>>(
           static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v), idx, counts,
-          static_cast<float*>(o), lse, s.B, s.N, s.H, block, nb, topk, scale);
+          static_cast<float*>(o), lse, s.B, s.N, s.H, bm, nb, topk, scale);
     return launch_status();
   }
 
   // bf16: tcgen05 tensor-core path
-  if (s.D != sol::attn100::kHeadDim || block != sol::attn100::kBlock) return SOL_ERR_UNSUPPORTED;
+  if (s.D != sol::attn100::kHeadDim || bm.block != sol::attn100::kBlock) return SOL_ERR_UNSUPPORTED;
   const long long tiles = static_cast<long long>(s.B) * s.H * nb;
   if (tiles > 0x7fffffffll) return SOL_ERR_UNSUPPORTED;
 #if SOL_ATTN_PINGPONG
-  {
+  if (bm.tw == 0) {
     CUtensorMap tq, tk, tv;
     if (sol_status st = make_bshd_map(&tq, q, s)) return st;
     if (sol_status st = make_bshd_map(&tk, k, s)) return st;
@@ -470,8 +546,13 @@ sol_status sparse_attn_impl(const void* q, const void* k, const void* v, const i
   }
 #endif
   CUtensorMap tk, tv;
-  if (sol_status st = make_bshd_map(&tk, k, s)) return st;
-  if (sol_status st = make_bshd_map(&tv, v, s)) return st;
+  if (bm.tw == 0) {
+    if (sol_status st = make_bshd_map(&tk, k, s)) return st;
+    if (sol_status st = make_bshd_map(&tv, v, s)) return st;
+  } else {
+    if (sol_status st = make_tile_map(&tk, k, s, bm)) return st;
+    if (sol_status st = make_tile_map(&tv, v, s, bm)) return st;
+  }
   const size_t smem = sizeof(sol::attn100::Smem) + 1024;
   if (!di->attn_attr) {
     if (cudaFuncSetAttribute(sol::attn100::sparse_attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -488,6 +569,8 @@ sol_status sparse_attn_impl(const void* q, const void* k, const void* v, const i
   p.B = s.B; p.N = s.N; p.H = s.H; p.nb = nb; p.topk = topk;
   p.num_tiles = static_cast<int>(tiles);
   p.scale_log2 = scale * 1.4426950408889634f;
+  p.bm = bm;
+  p.T = s.grid_t;
   const int grid = static_cast<int>(std::min<long long>(tiles, di->sm_count));
   sol::attn100::sparse_attn_fwd_kernel<<<grid, sol::attn100::kThreads, smem, stream>>>(tk, tv, p);
   return launch_status();

@@ -56,6 +56,16 @@ typedef struct {
   int grid_t, grid_h, grid_w;
 } sol_shape;
 
+/* 3-D token tiles (the *_tiled calls): block i is the tile (it, iy, ix) of
+ * t x h x w tokens, i = (it * (grid_h/h) + iy) * (grid_w/w) + ix, its tokens
+ * taken in raster order (frame, row, column) inside the tile; block = t*h*w.
+ * The tiles must cover the grid exactly (grid_t % t == grid_h % h ==
+ * grid_w % w == 0), else SOL_ERR_INVALID_ARG.  The pages leave the shape of
+ * the attention's "parts" open; runs of consecutive tokens are the default. */
+typedef struct {
+  int t, h, w;
+} sol_tile;
+
 /*
  * sol_qk_prologue -- fused QK-RMSNorm + 3D RoPE (normalisation and RoPE merged
  * into one kernel: ai-feiten.nl, "Videomodel MiniMax-H3 rendert sneller dan
@@ -142,7 +152,8 @@ sol_status sol_block_select_pooled(const float* qbar, const float* kbar, sol_sha
  *  SOL_SELECT_FORCE_DIAGONAL    every query block keeps its own key block i.
  *  SOL_SELECT_FORCE_FIRST_FRAME every query block keeps the key blocks that hold
  *                               tokens of frame t = 0: ids 0 .. ceil(grid_h *
- *                               grid_w / block) - 1.
+ *                               grid_w / block) - 1 (runs), or the first
+ *                               (grid_h/h)*(grid_w/w) ids (tiles).
  *  SOL_SELECT_TOP_P             the row keeps a mass-based count instead of a
  *                               fixed one (below).
  * A row's order is: forced blocks (ascending id), then the other blocks by
@@ -164,6 +175,10 @@ typedef struct {
   float top_p;             /* in (0, 1], read with SOL_SELECT_TOP_P         */
   float softmax_scale;     /* top-p softmax scale, <= 0: 1/sqrt(D)          */
   const int32_t* head_k;   /* NULL, or device int32 [H] per-head k          */
+  sol_tile tile;           /* {0,0,0}: blocks are runs of `block` tokens;
+                              else the means are of these tiles (t*h*w ==
+                              block) and the first-frame blocks are the
+                              (grid_h/h)*(grid_w/w) tiles of the first layer */
 } sol_select_opts;
 
 /*
@@ -215,6 +230,32 @@ sol_status sol_sparse_attn_fwd_counts(const void* q, const void* k, const void* 
                                       const int32_t* counts, sol_shape s, int block, int topk,
                                       float softmax_scale, sol_dtype dt, void* o, float* lse,
                                       cudaStream_t stream);
+
+/*
+ * sol_qk_prologue_pool_tiled -- sol_qk_prologue_pool with 3-D tile blocks:
+ * q_out, k_out are identical (tokens stay in place); qbar_out[b,h,i,:] is the
+ * fp32 mean of the stored q_out over the tokens of tile i, summed in the
+ * tile's raster order.  nb = N / (t*h*w).  Other arguments as
+ * sol_qk_prologue_pool.
+ */
+sol_status sol_qk_prologue_pool_tiled(const void* q_raw, const void* k_raw, void* q_out, void* k_out,
+                                      const float* gamma_q, const float* gamma_k, sol_shape s,
+                                      int rope_dt, int rope_dh, int rope_dw, float rope_theta, float eps,
+                                      sol_dtype dt, sol_tile tile, float* qbar_out, float* kbar_out,
+                                      cudaStream_t stream);
+
+/*
+ * sol_sparse_attn_fwd_tiled -- sol_sparse_attn_fwd (counts == NULL) or
+ * sol_sparse_attn_fwd_counts with 3-D tile blocks: the queries of tile i attend
+ * to the keys of the tiles idx[b,h,i,0..c-1].  Tokens stay in place in q, k,
+ * v and o (the kernel gathers each tile with one 5-D tensor-map copy); lse is
+ * [B,H,N] by token.  bf16: t*h*w == 128.  Other arguments as
+ * sol_sparse_attn_fwd_counts.
+ */
+sol_status sol_sparse_attn_fwd_tiled(const void* q, const void* k, const void* v, const int32_t* idx,
+                                     const int32_t* counts, sol_shape s, sol_tile tile, int topk,
+                                     float softmax_scale, sol_dtype dt, void* o, float* lse,
+                                     cudaStream_t stream);
 
 /*
  * sol_block_select_noalloc -- sol_block_select for callers that cannot

@@ -42,7 +42,7 @@ import numpy as np
 __all__ = [
     "bf16_round", "rope_angles", "qk_prologue", "block_pool", "block_scores",
     "topk_blocks", "near_tie_rows", "block_select", "sparse_attention",
-    "sparse_attention_rows", "selected_flops", "first_frame_blocks", "select_variant",
+    "sparse_attention_rows", "selected_flops", "first_frame_blocks", "select_variant", "tiled_blocks",
 ]
 
 
@@ -111,17 +111,49 @@ def qk_prologue(x, gamma, grid, split, theta: float, eps: float, tokens=None) ->
     return out
 
 
-def block_pool(x, block: int) -> np.ndarray:
-    """Mean of x over contiguous blocks of `block` tokens, float64 [B, H, nb, D].
+def tiled_blocks(grid, tile) -> list:
+    """Token ids of every 3-D tile block, a list of int arrays.
 
-    Reading: blocks are runs of consecutive raster-order tokens; the last block
-    may be short (N % block tokens) and is averaged over its valid tokens only.
+    The grid (T, Hg, Wg) is cut into tiles of tile = (t, h, w) tokens (exactly:
+    each extent divides the grid's); tiles are numbered in raster order of
+    their position (tile frame, tile row, tile column) and the tokens of a tile
+    are listed in raster order (frame, row, column).  Token ids are raster
+    order of the grid, n = (t * Hg + y) * Wg + x.
+    """
+    T, Hg, Wg = (int(g) for g in grid)
+    tt, th, tw = (int(x) for x in tile)
+    assert T % tt == 0 and Hg % th == 0 and Wg % tw == 0
+    blocks = []
+    for it in range(T // tt):
+        for iy in range(Hg // th):
+            for ix in range(Wg // tw):
+                ids = [((it * tt + dt) * Hg + iy * th + dy) * Wg + ix * tw + dx
+                       for dt in range(tt) for dy in range(th) for dx in range(tw)]
+                blocks.append(np.asarray(ids, dtype=np.int64))
+    return blocks
+
+
+def _members(N: int, block) -> list:
+    """Token ids of every block: `block` is a block size (runs of consecutive
+    tokens, the last one possibly short) or a list of id arrays (tiled_blocks)."""
+    if isinstance(block, (int, np.integer)):
+        return [np.arange(i * block, min(N, (i + 1) * block)) for i in range(-(-N // block))]
+    return list(block)
+
+
+def block_pool(x, block) -> np.ndarray:
+    """Mean of x over each block's tokens, float64 [B, H, nb, D].
+
+    Reading: by default blocks are runs of `block` consecutive raster-order
+    tokens; the last block may be short (N % block tokens) and is averaged over
+    its valid tokens only.  `block` may instead list each block's token ids
+    (3-D tiles: tiled_blocks).
     """
     B, N, H, D = x.shape
-    nb = -(-N // block)
-    out = np.empty((B, H, nb, D))
-    for i in range(nb):
-        seg = np.asarray(x[:, i * block:min(N, (i + 1) * block)], dtype=np.float64)   # [B, n_i, H, D]
+    members = _members(N, block)
+    out = np.empty((B, H, len(members), D))
+    for i, ids in enumerate(members):
+        seg = np.asarray(x[:, ids], dtype=np.float64)   # [B, n_i, H, D]
         out[:, :, i, :] = seg.mean(axis=1)
     return out
 
@@ -161,9 +193,13 @@ def block_select(q, k, block: int, topk: int):
     return topk_blocks(s, topk), s
 
 
-def first_frame_blocks(grid, block: int) -> int:
-    """Number of blocks holding a token of frame t = 0: tokens 0 .. grid_h * grid_w - 1
-    come first in raster order, so blocks 0 .. ceil(grid_h * grid_w / block) - 1."""
+def first_frame_blocks(grid, block: int, tile=None) -> int:
+    """Number of blocks holding a token of frame t = 0 (they are blocks 0 .. count - 1).
+    Runs: tokens 0 .. grid_h * grid_w - 1 come first in raster order, so
+    ceil(grid_h * grid_w / block).  Tiles (t, h, w): the tiles of the first
+    tile frame, (grid_h / h) * (grid_w / w)."""
+    if tile is not None:
+        return (int(grid[1]) // int(tile[1])) * (int(grid[2]) // int(tile[2]))
     return -(-(int(grid[1]) * int(grid[2])) // block)
 
 
@@ -212,7 +248,7 @@ def select_variant(scores, topk: int, *, diagonal: bool = False, first_blocks: i
     return idx, counts
 
 
-def sparse_attention_rows(q, k, v, idx, block: int, scale: float, b: int, h: int, i: int, count=None):
+def sparse_attention_rows(q, k, v, idx, block, scale: float, b: int, h: int, i: int, count=None):
     """Attention of the queries of block i of (b, h) over its kept key blocks.
 
     Keys: every token m < N of the blocks idx[b, h, i, :count] (all of the row
@@ -220,10 +256,10 @@ def sparse_attention_rows(q, k, v, idx, block: int, scale: float, b: int, h: int
     l_m = scale * q_n . k_m; two-pass softmax: subtract the row max, exponentiate,
     normalise.  Returns (o [n_i, D], lse [n_i]) with lse = ln sum_m exp(l_m).
     """
-    N = q.shape[1]
-    rows = np.arange(i * block, min(N, (i + 1) * block))
+    members = _members(q.shape[1], block)
+    rows = members[i]
     kept = np.asarray(idx[b, h, i])[:count]
-    cols = np.concatenate([np.arange(j * block, min(N, (j + 1) * block)) for j in kept])
+    cols = np.concatenate([members[j] for j in kept])
     qi = np.asarray(q[b, rows, h, :], np.float64)
     kj = np.asarray(k[b, cols, h, :], np.float64)
     vj = np.asarray(v[b, cols, h, :], np.float64)
@@ -236,12 +272,14 @@ def sparse_attention_rows(q, k, v, idx, block: int, scale: float, b: int, h: int
     return o, lse
 
 
-def sparse_attention(q, k, v, idx, block: int, scale: float | None = None, units=None, counts=None):
+def sparse_attention(q, k, v, idx, block, scale: float | None = None, units=None, counts=None):
     """Step a5 over all (b, h, query block) units, or over the listed `units`.
 
     q, k, v: [B, N, H, D] stored tensors (widened exactly to float64).
     idx: [B, H, nb, k] kept key-block ids; with counts [B, H, nb], row (b, h, i)
     keeps only its first counts[b, h, i] ids.  scale defaults to 1/sqrt(D).
+    block: block size (runs of consecutive tokens) or each block's token ids
+    (3-D tiles: tiled_blocks).
     Returns (o [B, N, H, D], lse [B, H, N]) float64; rows of units not computed
     are NaN.
     """
@@ -251,17 +289,16 @@ def sparse_attention(q, k, v, idx, block: int, scale: float | None = None, units
     B, N, H, D = q.shape
     if scale is None:
         scale = 1.0 / math.sqrt(D)
-    nb = -(-N // block)
+    members = _members(N, block)
     o = np.full((B, N, H, D), np.nan)
     lse = np.full((B, H, N), np.nan)
     if units is None:
-        units = [(b, h, i) for b in range(B) for h in range(H) for i in range(nb)]
+        units = [(b, h, i) for b in range(B) for h in range(H) for i in range(len(members))]
     for (b, h, i) in units:
         c = None if counts is None else int(counts[b, h, i])
-        oi, li = sparse_attention_rows(q, k, v, idx, block, scale, b, h, i, c)
-        r0, r1 = i * block, min(N, (i + 1) * block)
-        o[b, r0:r1, h, :] = oi
-        lse[b, h, r0:r1] = li
+        oi, li = sparse_attention_rows(q, k, v, idx, members, scale, b, h, i, c)
+        o[b, members[i], h, :] = oi
+        lse[b, h, members[i]] = li
     return o, lse
 
 

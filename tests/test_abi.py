@@ -150,9 +150,13 @@ def test_select_pooled_argument_checks(lib):
     assert f(FAKE, FAKE, big, 64, 4, FAKE, None, None) == UNSUPPORTED
 
 
+class TileStruct(ctypes.Structure):
+    _fields_ = [("t", ctypes.c_int), ("h", ctypes.c_int), ("w", ctypes.c_int)]
+
+
 class SelectOpts(ctypes.Structure):
     _fields_ = [("flags", ctypes.c_uint), ("top_p", ctypes.c_float), ("softmax_scale", ctypes.c_float),
-                ("head_k", ctypes.c_void_p)]
+                ("head_k", ctypes.c_void_p), ("tile", TileStruct)]
 
 
 def test_select_pooled_ex_argument_checks(lib):
@@ -188,3 +192,49 @@ def test_attention_counts_argument_checks(lib):
     assert f(FAKE, FAKE, FAKE, FAKE, FAKE, OK_SHAPE, 64, 0, 0.0, 0, FAKE, FAKE, None) == INVALID
     assert f(FAKE, FAKE, None, FAKE, FAKE, OK_SHAPE, 64, 4, 0.0, 0, FAKE, FAKE, None) == INVALID
     assert f(FAKE, FAKE, FAKE, FAKE, FAKE, OK_SHAPE, 64, 4, float("nan"), 0, FAKE, FAKE, None) == INVALID
+
+
+class Tile(ctypes.Structure):
+    _fields_ = [("t", ctypes.c_int), ("h", ctypes.c_int), ("w", ctypes.c_int)]
+
+
+def test_tiled_argument_checks(lib):
+    f = lib.sol_sparse_attn_fwd_tiled
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p] * 5 + [Shape, Tile, ctypes.c_int, ctypes.c_float, ctypes.c_int,
+                                          ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+    ok_tile = Tile(1, 8, 8)                       # 16 blocks of 64 on the 4x16x16 grid
+    assert f(FAKE, FAKE, FAKE, FAKE, None, OK_SHAPE, Tile(0, 8, 8), 4, 0.0, 0, FAKE, FAKE, None) == INVALID
+    assert f(FAKE, FAKE, FAKE, FAKE, None, OK_SHAPE, Tile(3, 8, 8), 4, 0.0, 0, FAKE, FAKE, None) == INVALID  # 4 % 3
+    assert f(FAKE, FAKE, FAKE, FAKE, None, OK_SHAPE, Tile(1, 5, 8), 4, 0.0, 0, FAKE, FAKE, None) == INVALID
+    assert f(FAKE, FAKE, FAKE, FAKE, None, OK_SHAPE, ok_tile, 17, 0.0, 0, FAKE, FAKE, None) == INVALID     # k > nb
+    assert f(FAKE, FAKE, None, FAKE, None, OK_SHAPE, ok_tile, 4, 0.0, 0, FAKE, FAKE, None) == INVALID
+    g = lib.sol_qk_prologue_pool_tiled
+    g.restype = ctypes.c_int
+    g.argtypes = [ctypes.c_void_p] * 6 + [Shape, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float,
+                                          ctypes.c_float, ctypes.c_int, Tile, ctypes.c_void_p, ctypes.c_void_p,
+                                          ctypes.c_void_p]
+
+    def call(tile=ok_tile, qbar=FAKE, split=(24, 20, 20)):
+        return g(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, OK_SHAPE, *split, 10000.0, 1e-6, 0, tile, qbar, FAKE, None)
+
+    assert call(tile=Tile(1, 16, 32)) == INVALID       # 16 % 32
+    assert call(tile=Tile(-1, 8, 8)) == INVALID
+    assert call(qbar=None) == INVALID
+    assert call(split=(24, 20, 18)) == INVALID
+
+
+def test_select_ex_tile_checks(lib):
+    f = lib.sol_block_select_pooled_ex
+    f.restype = ctypes.c_int
+
+    class Opts(ctypes.Structure):
+        _fields_ = [("flags", ctypes.c_uint), ("top_p", ctypes.c_float), ("softmax_scale", ctypes.c_float),
+                    ("head_k", ctypes.c_void_p), ("tile", Tile)]
+
+    f.argtypes = [ctypes.c_void_p, ctypes.c_void_p, Shape, ctypes.c_int, ctypes.c_int, ctypes.POINTER(Opts),
+                  ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+    bad = Opts(2, 1.0, 0.0, None, Tile(1, 8, 4))       # 32 tokens per tile, but block 64
+    assert f(FAKE, FAKE, OK_SHAPE, 64, 4, ctypes.byref(bad), FAKE, FAKE, None, None) == INVALID
+    bad2 = Opts(2, 1.0, 0.0, None, Tile(1, 3, 8))      # does not divide the grid
+    assert f(FAKE, FAKE, OK_SHAPE, 64, 4, ctypes.byref(bad2), FAKE, FAKE, None, None) == INVALID

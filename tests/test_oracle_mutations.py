@@ -13,6 +13,7 @@ import pytest
 import oracle
 import oracle.sol_oracle as so
 from tests import test_oracle_pins as pins
+from tests import test_oracle_tiles as tpins
 from tests import test_oracle_variants as vpins
 
 
@@ -76,9 +77,9 @@ def _attention_rows_no_scale(q, k, v, idx, block, scale, b, h, i, count=None):
 
 def _attention_rows_lse_no_max(q, k, v, idx, block, scale, b, h, i, count=None):
     o, lse = so.__dict__["_orig_rows"](q, k, v, idx, block, scale, b, h, i, count)
-    N = q.shape[1]
-    rows = np.arange(i * block, min(N, (i + 1) * block))
-    cols = np.concatenate([np.arange(j * block, min(N, (j + 1) * block)) for j in np.asarray(idx[b, h, i])[:count]])
+    members = so._members(q.shape[1], block)
+    rows = members[i]
+    cols = np.concatenate([members[j] for j in np.asarray(idx[b, h, i])[:count]])
     logits = scale * (np.asarray(q[b, rows, h], np.float64) @ np.asarray(k[b, cols, h], np.float64).T)
     mx = logits.max(axis=1)
     return o, lse - mx
@@ -96,6 +97,10 @@ def _variant_head_k_ignored(scores, topk, **kw):
     return so.__dict__["_orig_variant"](scores, topk, **{**kw, "head_k": None})
 
 
+def _tiles_rows_columns_swapped(grid, tile):
+    return so.__dict__["_orig_tiles"](grid, (tile[0], tile[2], tile[1]))
+
+
 MUTATIONS = [
     ("qk_prologue", _prologue_rope_sign, [pins.test_prologue_hand_case]),
     ("rope_angles", _angles_axis_reversed, [pins.test_prologue_hand_case]),
@@ -108,6 +113,7 @@ MUTATIONS = [
     ("select_variant", _variant_diagonal_dropped, [lambda: vpins.test_forced_diagonal_brute_force(2)]),
     ("select_variant", _variant_scale_ignored, [lambda: vpins.test_top_p_count_is_smallest_subset_reaching_p(0.6)]),
     ("select_variant", _variant_head_k_ignored, [vpins.test_per_head_k]),
+    ("tiled_blocks", _tiles_rows_columns_swapped, [tpins.test_tiled_blocks_hand_case]),
 ]
 
 
@@ -115,6 +121,7 @@ MUTATIONS = [
 def test_pins_catch_planted_mistake(monkeypatch, name, bad, tests):
     monkeypatch.setitem(so.__dict__, "_orig_rows", so.sparse_attention_rows)
     monkeypatch.setitem(so.__dict__, "_orig_variant", so.select_variant)
+    monkeypatch.setitem(so.__dict__, "_orig_tiles", so.tiled_blocks)
     monkeypatch.setattr(so, name, bad)
     monkeypatch.setattr(oracle, name, bad)
     for t in tests:
