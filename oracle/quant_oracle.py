@@ -1,0 +1,86 @@
+"""Oracle of the quantised token <-> head exchange around the Sol-Attn path.
+
+TEST INFRASTRUCTURE ONLY (like sol_oracle): imported by tests/ and nothing in
+the product path.  It shares no code with the CUDA path.
+
+Source.  For multi-GPU runs the Sol-H3 runtime moves Q, K and V between GPUs
+as INT8 and the attention output as FP8, cutting inter-GPU traffic by about a
+half (ai-feiten.nl, "Videomodel MiniMax-H3 rendert sneller dan afspelen",
+section "Waar de snelheidswinst vandaan komt").  The pages give no format
+details; the readings written out here are:
+
+  - one scale per (token, head) row of D channels, symmetric, in fp32:
+    s = max_d |x_d| / L with L = 127 (INT8) or 448 (FP8 e4m3, its largest
+    finite value); a row of zeros gets s = 0 and all-zero codes;
+  - INT8 code = clamp(round_half_even(x / s), -127, 127); e4m3 code = x / s
+    rounded to the nearest e4m3 value (ties to even), saturating at +-448;
+    the quotient x / s is one IEEE fp32 division, and max, division and
+    rounding decide the code in fp32 exactly as written;
+  - dequantised value = bf16_round(fp32(code * s)).
+  - sequence-parallel layout: G ranks; rank r owns tokens [r N/G, (r+1) N/G)
+    of all heads before the attention and heads [r H/G, (r+1) H/G) of all
+    tokens during it.  Because every scale belongs to one (token, head) row,
+    the quantised values do not depend on G.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from .sol_oracle import bf16_round
+
+__all__ = ["INT8_LEVELS", "E4M3_MAX", "e4m3_round", "quantize_rows", "dequantize_rows", "quant_roundtrip"]
+
+INT8_LEVELS = 127.0
+E4M3_MAX = 448.0
+
+
+def e4m3_round(x) -> np.ndarray:
+    """Nearest FP8 e4m3 value (ties to even), saturating at +-448; float64 result.
+
+    e4m3: 1 sign, 4 exponent bits (bias 7), 3 mantissa bits, no infinities.
+    Normal numbers m * 2^e with 1 <= m < 2 and e >= -6 are spaced 2^(e-3);
+    below 2^-6 the subnormals are spaced 2^-9.  The largest finite value is
+    1.75 * 2^8 = 448.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    a = np.abs(x)
+    _, fe = np.frexp(a)                           # a = f * 2^fe, 0.5 <= f < 1: exponent fe - 1
+    e = np.maximum(fe.astype(np.float64) - 1.0, -6.0)   # subnormal range keeps the 2^-9 spacing
+    step = np.exp2(e - 3.0)
+    r = np.rint(a / step) * step                  # np.rint: half to even (in units of the step)
+    r = np.minimum(r, E4M3_MAX)
+    return np.copysign(r, x)
+
+
+def quantize_rows(x, kind: str):
+    """Codes and scales of rows x[..., D] (stored bf16 / fp32 values).
+
+    kind "int8" or "e4m3".  Returns (codes float64 [..., D] holding the code
+    values, scales float32 [...]).
+    """
+    x32 = np.asarray(x, dtype=np.float32)
+    levels = np.float32(INT8_LEVELS if kind == "int8" else E4M3_MAX)
+    amax = np.max(np.abs(x32), axis=-1)
+    s = (amax / levels).astype(np.float32)                       # one fp32 division
+    safe = np.where(s > 0, s, np.float32(1.0)).astype(np.float32)
+    quo = (x32 / safe[..., None]).astype(np.float32)             # one fp32 division per value
+    if kind == "int8":
+        codes = np.clip(np.rint(quo.astype(np.float64)), -127.0, 127.0)
+    elif kind == "e4m3":
+        codes = e4m3_round(quo.astype(np.float64))
+    else:
+        raise ValueError(kind)
+    codes = np.where(s[..., None] > 0, codes, 0.0)
+    return codes, s
+
+
+def dequantize_rows(codes, scales) -> np.ndarray:
+    """bf16_round(fp32(code * s)), float64 result."""
+    prod = np.asarray(codes, np.float32) * np.asarray(scales, np.float32)[..., None]
+    return bf16_round(prod.astype(np.float32).astype(np.float64))
+
+
+def quant_roundtrip(x, kind: str) -> np.ndarray:
+    """The values a tensor [..., D] arrives with after quantisation and dequantisation."""
+    codes, s = quantize_rows(x, kind)
+    return dequantize_rows(codes, s)

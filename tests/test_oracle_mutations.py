@@ -13,6 +13,7 @@ import pytest
 import oracle
 import oracle.sol_oracle as so
 from tests import test_oracle_pins as pins
+from tests import test_oracle_quant as qpins
 from tests import test_oracle_tiles as tpins
 from tests import test_oracle_variants as vpins
 
@@ -101,6 +102,19 @@ def _tiles_rows_columns_swapped(grid, tile):
     return so.__dict__["_orig_tiles"](grid, (tile[0], tile[2], tile[1]))
 
 
+def _e4m3_no_subnormals(x):
+    x = np.asarray(x, dtype=np.float64)
+    a = np.abs(x)
+    _, fe = np.frexp(a)
+    step = np.exp2(fe.astype(np.float64) - 4.0)         # normal spacing all the way down
+    return np.copysign(np.minimum(np.rint(a / step) * step, 448.0), x)
+
+
+def _quantize_levels_128(x, kind):
+    codes, s = oracle.quant_oracle.__dict__["_orig_quant"](x, kind)
+    return codes, (s * np.float32(127.0) / np.float32(128.0)).astype(np.float32)
+
+
 MUTATIONS = [
     ("qk_prologue", _prologue_rope_sign, [pins.test_prologue_hand_case]),
     ("rope_angles", _angles_axis_reversed, [pins.test_prologue_hand_case]),
@@ -114,6 +128,8 @@ MUTATIONS = [
     ("select_variant", _variant_scale_ignored, [lambda: vpins.test_top_p_count_is_smallest_subset_reaching_p(0.6)]),
     ("select_variant", _variant_head_k_ignored, [vpins.test_per_head_k]),
     ("tiled_blocks", _tiles_rows_columns_swapped, [tpins.test_tiled_blocks_hand_case]),
+    ("e4m3_round", _e4m3_no_subnormals, [qpins.test_e4m3_round_matches_torch]),
+    ("quantize_rows", _quantize_levels_128, [qpins.test_scales_and_dequantize_hand_case]),
 ]
 
 
@@ -122,7 +138,8 @@ def test_pins_catch_planted_mistake(monkeypatch, name, bad, tests):
     monkeypatch.setitem(so.__dict__, "_orig_rows", so.sparse_attention_rows)
     monkeypatch.setitem(so.__dict__, "_orig_variant", so.select_variant)
     monkeypatch.setitem(so.__dict__, "_orig_tiles", so.tiled_blocks)
-    monkeypatch.setattr(so, name, bad)
+    monkeypatch.setitem(oracle.quant_oracle.__dict__, "_orig_quant", oracle.quant_oracle.quantize_rows)
+    monkeypatch.setattr(so, name, bad, raising=False)
     monkeypatch.setattr(oracle, name, bad)
     for t in tests:
         with pytest.raises(AssertionError):
