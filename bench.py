@@ -426,6 +426,92 @@ def run_ours(args, wl, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------- sequence-parallel arm (opt-in)
+def run_seqpar(args, wl, world, rank, local):
+    """One clip over `world` ranks: each rank holds a token shard, the attention runs on
+    head shards behind an INT8 Q/K/V and FP8 O all-to-all (strong scaling).  With one
+    rank the exchange is a local copy and the line measures the quantisation kernels
+    and the chain on quantised inputs."""
+    import block_sparse_attention_sol_b200 as sol  # noqa: F401  (loads libsol)
+    from block_sparse_attention_sol_b200.seqpar import CollectiveTransport, LocalTransport, SeqParallelAttention
+    topk = wl.topk[0]
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    inp = make_inputs(wl, seed=0)
+    nl = wl.N // world
+    shard = {n: inp[n][:, rank * nl:(rank + 1) * nl].contiguous().to(dev) for n in ("q", "k", "v")}
+    gq, gk = inp["gamma_q"].to(dev), inp["gamma_k"].to(dev)
+    sp = SeqParallelAttention(rank, world, wl.B, wl.N, wl.H, wl.D, wl.grid, wl.block, topk, gq, gk, wl.rope_split,
+                              wl.rope_theta, wl.eps, device=dev)
+    transport = LocalTransport() if world == 1 else CollectiveTransport()
+    out = torch.empty_like(shard["q"])
+
+    def step(ev=None):
+        marks = []
+        def mark():
+            if ev is not None:
+                ev[len(marks)].record(stream)
+            marks.append(0)
+        mark()
+        sp.stage_pack(shard["q"], shard["k"], shard["v"])
+        mark()
+        sp.exchange_qkv(transport)
+        mark()
+        sp.stage_compute()
+        mark()
+        sp.exchange_o(transport)
+        mark()
+        sp.stage_unpack(out)
+        mark()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    with sampler:
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        start.record(stream)
+        for s_ in range(args.steps):
+            step(evs[s_])
+        stop.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+    if sol.sol_check_device_status() != sol.SOL_OK:
+        raise RuntimeError("device-side error in the timed region")
+    ms = max_over_ranks(start.elapsed_time(stop) / args.steps, world)
+    names = ("pack_qkv", "exchange_qkv", "compute", "exchange_o", "unpack_o")
+    st = {n: sum(e[i].elapsed_time(e[i + 1]) for e in evs) / args.steps for i, n in enumerate(names)}
+    flops = wl.selected_flops(topk)
+    peaks = load_peaks()
+    p = sp.plan
+    rows_in = wl.B * nl * wl.H                       # this rank's token-shard rows per tensor
+    pack_b = 3 * rows_in * (wl.D * 2 + wl.D + 4)     # read bf16, write codes + scale
+    unpack_qkv_b = 3 * p.G * p.rows * (wl.D + 4 + wl.D * 2)
+    clocks = sampler.summary()
+    if rank != 0:
+        return
+    line = {
+        "metric": "sparse-attn effective TFLOP/s (selected FLOPs)", "value": flops / (ms * 1e-3) / 1e12,
+        "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "config_id": wl.config_id, "B": wl.B, "N": wl.N, "H": wl.H, "D": wl.D,
+                   "grid": list(wl.grid), "block": wl.block, "topk": topk,
+                   "parallelism": f"sequence-parallel x{world}: INT8 Q/K/V and FP8 O all-to-all "
+                                  f"({'local copy' if world == 1 else 'NCCL'})"},
+        "stages_ms": st,
+        "pack_qkv": {"GB/s": pack_b / st["pack_qkv"] / 1e6, "frac_hbm": pack_b / st["pack_qkv"] / 1e6 / peaks["hbm_gbs"]},
+        "wire_bytes_per_rank": p.wire_bytes(), "bf16_wire_bytes_per_rank": p.bf16_wire_bytes(),
+        "unpack_qkv_bytes": unpack_qkv_b,
+        "gpu_launches": 11 * args.steps,       # 3 packs, 3 unpacks, the 3-kernel chain, O pack + unpack
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -441,6 +527,9 @@ def main():
     ap.add_argument("--chain", choices=("fused", "split"), default="fused",
                     help="fused: prologue emits the block means (3 launches per step); split: the selection "
                          "pools q and k itself (4 launches)")
+    ap.add_argument("--parallel", choices=("clips", "seqpar"), default="clips",
+                    help="clips: an independent clip per rank (default); seqpar: one clip over all ranks with "
+                         "a quantised all-to-all around the path")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -451,6 +540,8 @@ def main():
     try:
         if args.impl == "reference":
             run_reference(args, wl, world, rank)
+        elif args.parallel == "seqpar":
+            run_seqpar(args, wl, world, rank, local)
         else:
             run_ours(args, wl, world, rank, local)
     finally:

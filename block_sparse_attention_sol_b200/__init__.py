@@ -15,6 +15,8 @@ Functions (same names as the C ABI):
     sol_sparse_attn_fwd_counts(q, k, v, idx, counts, grid, block, ...) -> (o, lse)
     sol_qk_prologue_pool_tiled(q_raw, k_raw, gamma_q, gamma_k, grid, tile, ...) -> (q, k, qbar, kbar)
     sol_sparse_attn_fwd_tiled(q, k, v, idx, grid, tile, counts=None, ...) -> (o, lse)
+    sol_quant_pack(x, G, split, code, codes_out, scales_out, ...)  (exchange buffers)
+    sol_dequant_unpack(codes, scales, B, Nc, Hc, D, G, split, code, out, ...)
     sol_check_device_status(stream=None)
     sol_selftest_wait_timeout(limit_us, stream=None)
     sol_block_select_workspace_bytes(shape, block)
@@ -30,7 +32,8 @@ __all__ = [
     "SolError", "SolShape", "LIB_PATH", "lib",
     "sol_qk_prologue", "sol_block_select", "sol_block_select_workspace_bytes", "sol_sparse_attn_fwd",
     "sol_qk_prologue_pool", "sol_block_select_pooled", "sol_block_select_pooled_ex", "sol_sparse_attn_fwd_counts",
-    "SolSelectOpts", "SolTile", "sol_qk_prologue_pool_tiled", "sol_sparse_attn_fwd_tiled", "SOL_SELECT_FORCE_DIAGONAL", "SOL_SELECT_FORCE_FIRST_FRAME", "SOL_SELECT_TOP_P",
+    "SolSelectOpts", "SolTile", "sol_quant_pack", "sol_dequant_unpack",
+    "SOL_CODE_INT8", "SOL_CODE_E4M3", "SOL_SPLIT_HEADS", "SOL_SPLIT_TOKENS", "sol_qk_prologue_pool_tiled", "sol_sparse_attn_fwd_tiled", "SOL_SELECT_FORCE_DIAGONAL", "SOL_SELECT_FORCE_FIRST_FRAME", "SOL_SELECT_TOP_P",
     "sol_check_device_status", "sol_selftest_wait_timeout", "sol_status_string", "sol_attention_chain",
     "SOL_OK", "SOL_ERR_INVALID_ARG", "SOL_ERR_UNSUPPORTED", "SOL_ERR_CUDA", "SOL_ERR_TIMEOUT",
 ]
@@ -45,6 +48,8 @@ lib = ctypes.CDLL(LIB_PATH)
 SOL_OK, SOL_ERR_INVALID_ARG, SOL_ERR_UNSUPPORTED, SOL_ERR_CUDA, SOL_ERR_TIMEOUT = range(5)
 SOL_F32, SOL_BF16 = 0, 1
 SOL_SELECT_FORCE_DIAGONAL, SOL_SELECT_FORCE_FIRST_FRAME, SOL_SELECT_TOP_P = 1, 2, 4
+SOL_CODE_INT8, SOL_CODE_E4M3 = 0, 1
+SOL_SPLIT_HEADS, SOL_SPLIT_TOKENS = 0, 1
 
 
 class SolShape(ctypes.Structure):
@@ -88,6 +93,10 @@ lib.sol_qk_prologue_pool_tiled.argtypes = [_P, _P, _P, _P, _P, _P, SolShape, _I,
                                            _P]
 lib.sol_sparse_attn_fwd_tiled.restype = _I
 lib.sol_sparse_attn_fwd_tiled.argtypes = [_P, _P, _P, _P, _P, SolShape, SolTile, _I, _F, _I, _P, _P, _P]
+lib.sol_quant_pack.restype = _I
+lib.sol_quant_pack.argtypes = [_P, _I, _I, _I, _I, _I, _I, _I, _P, _P, ctypes.c_longlong, _P]
+lib.sol_dequant_unpack.restype = _I
+lib.sol_dequant_unpack.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _I, _P, ctypes.c_longlong, _P]
 lib.sol_sparse_attn_fwd.restype = _I
 lib.sol_sparse_attn_fwd.argtypes = [_P, _P, _P, _P, SolShape, _I, _I, _F, _I, _P, _P, _P]
 lib.sol_check_device_status.restype = _I
@@ -325,6 +334,30 @@ def sol_sparse_attn_fwd_tiled(q, k, v, idx, grid, tile, counts=None, softmax_sca
                                        _dtype_code(q), o.data_ptr(), lse.data_ptr(), _stream_handle(stream))
     _check(st, "sol_sparse_attn_fwd_tiled")
     return o, lse
+
+
+def sol_quant_pack(x, G, split, code, codes_out, scales_out, g_stride_rows=0, stream=None):
+    """Quantise bf16 rows x [B, N, H, D] into per-destination slices (see include/sol.h).
+    codes_out (uint8) and scales_out (float32) are caller buffers, slice g at row g * g_stride_rows."""
+    _cuda(x, "x")
+    if x.dtype != torch.bfloat16 or x.dim() != 4:
+        raise TypeError("x must be bf16 [B, N, H, D]")
+    if codes_out.dtype != torch.uint8 or scales_out.dtype != torch.float32:
+        raise TypeError("codes_out must be uint8 and scales_out float32")
+    B, N, H, D = x.shape
+    st = lib.sol_quant_pack(x.data_ptr(), B, N, H, D, int(G), int(split), int(code), _cuda(codes_out, "codes_out").data_ptr(),
+                            _cuda(scales_out, "scales_out").data_ptr(), int(g_stride_rows), _stream_handle(stream))
+    _check(st, "sol_quant_pack")
+
+
+def sol_dequant_unpack(codes, scales, B, Nc, Hc, D, G, split, code, out, g_stride_rows=0, stream=None):
+    """Dequantise G received slices into bf16 out (tokens or heads concatenated; see include/sol.h)."""
+    _cuda(codes, "codes"), _cuda(scales, "scales"), _cuda(out, "out")
+    if out.dtype != torch.bfloat16:
+        raise TypeError("out must be bf16")
+    st = lib.sol_dequant_unpack(codes.data_ptr(), scales.data_ptr(), int(B), int(Nc), int(Hc), int(D), int(G), int(split),
+                                int(code), out.data_ptr(), int(g_stride_rows), _stream_handle(stream))
+    _check(st, "sol_dequant_unpack")
 
 
 def sol_check_device_status(stream=None) -> int:

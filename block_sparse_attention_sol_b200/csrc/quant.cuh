@@ -1,0 +1,137 @@
+// Quantised exchange buffers for sequence-parallel Sol-Attn.
+//
+// Multi-GPU runs of the Sol-H3 runtime move Q, K and V between GPUs as INT8 and
+// the attention output as FP8, halving the inter-GPU bytes (ai-feiten.nl,
+// "Videomodel MiniMax-H3 rendert sneller dan afspelen", section "Waar de
+// snelheidswinst vandaan komt").  Here a row is the D channels of one
+// (batch, token, head); each row gets one fp32 scale s = max|x| / L
+// (L = 127 for INT8, 448 for e4m3) and codes x / s rounded to nearest even
+// (INT8 clamped to +-127, e4m3 saturating), all decided in fp32.
+//
+//   quant_pack:     bf16 rows [B, N, H, D] -> codes + scales packed by
+//                   destination rank g: [G][B][Nc][Hc][D] and [G][B][Nc][Hc].
+//                   Split heads (token shard -> head shards): Hc = H / G,
+//                   Nc = N, g = h / Hc.  Split tokens (head shard -> token
+//                   shards): Nc = N / G, Hc = H, g = n / Nc.
+//   dequant_unpack: codes + scales [G][B][Nc][Hc] received from G ranks ->
+//                   bf16 bf16_rn(code * s), concatenated along tokens (the
+//                   slices were head shards of token shards) or along heads.
+// Both are HBM streams: D / 8 lanes per row, 16-byte bf16 loads / stores and
+// 8-byte code stores / loads.  Slice g starts g * g_stride rows into the
+// buffers, so several tensors can share one exchange buffer.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <cstdint>
+
+namespace sol {
+namespace quant {
+
+enum : int { kSplitHeads = 0, kSplitTokens = 1 };
+enum : int { kInt8 = 0, kE4M3 = 1 };
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4 w, float (&v)[8]) {
+  const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[2 * i] = __uint_as_float(u[i] << 16);
+    v[2 * i + 1] = __uint_as_float(u[i] & 0xFFFF0000u);
+  }
+}
+
+template <int CODE>
+__device__ __forceinline__ uint8_t encode(float q) {
+  if constexpr (CODE == kInt8) {
+    const int c = min(max(__float2int_rn(q), -127), 127);
+    return static_cast<uint8_t>(static_cast<int8_t>(c));
+  } else {
+    return static_cast<uint8_t>(__nv_cvt_float_to_fp8(q, __NV_SATFINITE, __NV_E4M3));
+  }
+}
+
+template <int CODE>
+__device__ __forceinline__ float decode(uint8_t c) {
+  if constexpr (CODE == kInt8) {
+    return static_cast<float>(static_cast<int8_t>(c));
+  } else {
+    const __half_raw h = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(c), __NV_E4M3);
+    return __half2float(__half(h));
+  }
+}
+
+// Thread t handles channels 8 (t % L) .. +7 of row t / L, L = D / 8.
+template <int D, int CODE>
+__global__ void __launch_bounds__(256) quant_pack_kernel(const __nv_bfloat16* __restrict__ x,
+                                                         uint8_t* __restrict__ codes, float* __restrict__ scales,
+                                                         int B, int N, int H, int G, int split, long long g_stride) {
+  constexpr int L = D / 8;
+  const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const long long row = gid / L;
+  const int li = static_cast<int>(gid % L);
+  if (row >= static_cast<long long>(B) * N * H) return;   // a row's L lanes leave together
+  const unsigned lane = threadIdx.x & 31u;
+  const unsigned seg = (L == 32) ? 0xffffffffu : (((1u << L) - 1u) << (lane & ~static_cast<unsigned>(L - 1)));
+
+  float v[8];
+  bf16x8_to_f32(__ldcs(reinterpret_cast<const uint4*>(x + row * D + li * 8)), v);
+  float a = 0.f;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) a = fmaxf(a, fabsf(v[e]));
+#pragma unroll
+  for (int o = L / 2; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(seg, a, o));
+  const float s = __fdiv_rn(a, CODE == kInt8 ? 127.0f : 448.0f);
+
+  const int h = static_cast<int>(row % H);
+  const long long bn = row / H;
+  const int n = static_cast<int>(bn % N);
+  const int b = static_cast<int>(bn / N);
+  int g, nc, hc, Nc, Hc;
+  if (split == kSplitHeads) { Hc = H / G; Nc = N; g = h / Hc; hc = h % Hc; nc = n; }
+  else { Nc = N / G; Hc = H; g = n / Nc; nc = n % Nc; hc = h; }
+  const long long drow = g * g_stride + (static_cast<long long>(b) * Nc + nc) * Hc + hc;
+
+  uint32_t w[2] = {0u, 0u};
+  if (s > 0.f) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) w[e >> 2] |= static_cast<uint32_t>(encode<CODE>(__fdiv_rn(v[e], s))) << (8 * (e & 3));
+  }
+  __stcs(reinterpret_cast<uint2*>(codes + drow * D + li * 8), make_uint2(w[0], w[1]));
+  if (li == 0) scales[drow] = s;
+}
+
+template <int D, int CODE>
+__global__ void __launch_bounds__(256) dequant_unpack_kernel(const uint8_t* __restrict__ codes,
+                                                             const float* __restrict__ scales,
+                                                             __nv_bfloat16* __restrict__ out, int B, int Nc, int Hc,
+                                                             int G, int split, long long g_stride) {
+  constexpr int L = D / 8;
+  const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const long long row = gid / L;   // over [G][B][Nc][Hc]
+  const int li = static_cast<int>(gid % L);
+  const long long per_g = static_cast<long long>(B) * Nc * Hc;
+  if (row >= G * per_g) return;
+  const int g = static_cast<int>(row / per_g);
+  const long long r = row % per_g;
+  const int hc = static_cast<int>(r % Hc);
+  const int nc = static_cast<int>((r / Hc) % Nc);
+  const int b = static_cast<int>(r / (static_cast<long long>(Hc) * Nc));
+  const long long srow = g * g_stride + r;
+  const float s = __ldg(scales + srow);
+  const uint2 c = __ldcs(reinterpret_cast<const uint2*>(codes + srow * D + li * 8));
+  const uint32_t cw[2] = {c.x, c.y};
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float lo = __fmul_rn(decode<CODE>(static_cast<uint8_t>(cw[i >> 1] >> (16 * (i & 1)))), s);
+    const float hi = __fmul_rn(decode<CODE>(static_cast<uint8_t>(cw[i >> 1] >> (16 * (i & 1) + 8))), s);
+    const __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+    o[i] = *reinterpret_cast<const uint32_t*>(&p);
+  }
+  long long orow;
+  if (split == kSplitHeads) orow = (static_cast<long long>(b) * G * Nc + static_cast<long long>(g) * Nc + nc) * Hc + hc;
+  else orow = (static_cast<long long>(b) * Nc + nc) * (static_cast<long long>(G) * Hc) + static_cast<long long>(g) * Hc + hc;
+  __stcs(reinterpret_cast<uint4*>(out + orow * D + li * 8), make_uint4(o[0], o[1], o[2], o[3]));
+}
+
+}  // namespace quant
+}  // namespace sol

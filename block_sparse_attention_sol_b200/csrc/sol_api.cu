@@ -23,6 +23,7 @@
 #include "prologue.cuh"
 #include "select.cuh"
 #include "attn_pp.cuh"
+#include "quant.cuh"
 
 #ifndef SOL_ATTN_PINGPONG
 #define SOL_ATTN_PINGPONG 0   // 1: two query tiles per CTA in ping-pong (attn_pp.cuh)
@@ -452,6 +453,77 @@ sol_status sol_block_select_pooled_ex(const float* qbar, const float* kbar, sol_
   const float scale = opts->softmax_scale > 0.f ? opts->softmax_scale : 1.0f / std::sqrt(static_cast<float>(s.D));
   a.scale_log2 = scale * 1.4426950408889634f;   // log2(e)
   return launch_score_topk(di, s.D, plan, stream, qbar, kbar, a);
+}
+
+sol_status sol_quant_pack(const void* x, int B, int N, int H, int D, int G, sol_split split, sol_code code,
+                          void* codes_out, float* scales_out, long long g_stride_rows, cudaStream_t stream) {
+  if (!x || !codes_out || !scales_out) return SOL_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(codes_out) || reinterpret_cast<uintptr_t>(scales_out) % 4) return SOL_ERR_INVALID_ARG;
+  if (B < 1 || N < 1 || H < 1 || G < 1) return SOL_ERR_INVALID_ARG;
+  if (split != SOL_SPLIT_HEADS && split != SOL_SPLIT_TOKENS) return SOL_ERR_INVALID_ARG;
+  if (code != SOL_CODE_INT8 && code != SOL_CODE_E4M3) return SOL_ERR_INVALID_ARG;
+  if ((split == SOL_SPLIT_HEADS ? H : N) % G != 0) return SOL_ERR_INVALID_ARG;
+  const long long per_g = static_cast<long long>(B) * N * H / G;
+  if (g_stride_rows == 0) g_stride_rows = per_g;
+  if (g_stride_rows < per_g) return SOL_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return SOL_ERR_UNSUPPORTED;
+  const long long threads = static_cast<long long>(B) * N * H * (D / 8);
+  const long long grid = (threads + 255) / 256;
+  if (grid > 0x7fffffffll) return SOL_ERR_UNSUPPORTED;
+  const auto* xb = static_cast<const __nv_bfloat16*>(x);
+  auto* cb = static_cast<uint8_t*>(codes_out);
+  const dim3 g(static_cast<unsigned>(grid));
+  if (D == 128) {
+    if (code == SOL_CODE_INT8)
+      sol::quant::quant_pack_kernel<128, sol::quant::kInt8><<<g, 256, 0, stream>>>(xb, cb, scales_out, B, N, H, G, split,
+                                                                                   g_stride_rows);
+    else
+      sol::quant::quant_pack_kernel<128, sol::quant::kE4M3><<<g, 256, 0, stream>>>(xb, cb, scales_out, B, N, H, G, split,
+                                                                                   g_stride_rows);
+  } else {
+    if (code == SOL_CODE_INT8)
+      sol::quant::quant_pack_kernel<64, sol::quant::kInt8><<<g, 256, 0, stream>>>(xb, cb, scales_out, B, N, H, G, split,
+                                                                                  g_stride_rows);
+    else
+      sol::quant::quant_pack_kernel<64, sol::quant::kE4M3><<<g, 256, 0, stream>>>(xb, cb, scales_out, B, N, H, G, split,
+                                                                                  g_stride_rows);
+  }
+  return launch_status();
+}
+
+sol_status sol_dequant_unpack(const void* codes, const float* scales, int B, int Nc, int Hc, int D, int G,
+                              sol_split split, sol_code code, void* out, long long g_stride_rows, cudaStream_t stream) {
+  if (!codes || !scales || !out) return SOL_ERR_INVALID_ARG;
+  if (!aligned16(codes) || !aligned16(out) || reinterpret_cast<uintptr_t>(scales) % 4) return SOL_ERR_INVALID_ARG;
+  if (B < 1 || Nc < 1 || Hc < 1 || G < 1) return SOL_ERR_INVALID_ARG;
+  if (split != SOL_SPLIT_HEADS && split != SOL_SPLIT_TOKENS) return SOL_ERR_INVALID_ARG;
+  if (code != SOL_CODE_INT8 && code != SOL_CODE_E4M3) return SOL_ERR_INVALID_ARG;
+  const long long per_g = static_cast<long long>(B) * Nc * Hc;
+  if (g_stride_rows == 0) g_stride_rows = per_g;
+  if (g_stride_rows < per_g) return SOL_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return SOL_ERR_UNSUPPORTED;
+  const long long threads = G * per_g * (D / 8);
+  const long long grid = (threads + 255) / 256;
+  if (grid > 0x7fffffffll) return SOL_ERR_UNSUPPORTED;
+  const auto* cb = static_cast<const uint8_t*>(codes);
+  auto* ob = static_cast<__nv_bfloat16*>(out);
+  const dim3 g(static_cast<unsigned>(grid));
+  if (D == 128) {
+    if (code == SOL_CODE_INT8)
+      sol::quant::dequant_unpack_kernel<128, sol::quant::kInt8><<<g, 256, 0, stream>>>(cb, scales, ob, B, Nc, Hc, G,
+                                                                                       split, g_stride_rows);
+    else
+      sol::quant::dequant_unpack_kernel<128, sol::quant::kE4M3><<<g, 256, 0, stream>>>(cb, scales, ob, B, Nc, Hc, G,
+                                                                                       split, g_stride_rows);
+  } else {
+    if (code == SOL_CODE_INT8)
+      sol::quant::dequant_unpack_kernel<64, sol::quant::kInt8><<<g, 256, 0, stream>>>(cb, scales, ob, B, Nc, Hc, G,
+                                                                                      split, g_stride_rows);
+    else
+      sol::quant::dequant_unpack_kernel<64, sol::quant::kE4M3><<<g, 256, 0, stream>>>(cb, scales, ob, B, Nc, Hc, G,
+                                                                                      split, g_stride_rows);
+  }
+  return launch_status();
 }
 
 sol_status sol_sparse_attn_fwd(const void* q, const void* k, const void* v, const int32_t* idx, sol_shape s,

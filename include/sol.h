@@ -258,6 +258,40 @@ sol_status sol_sparse_attn_fwd_tiled(const void* q, const void* k, const void* v
                                      cudaStream_t stream);
 
 /*
+ * Quantised exchange buffers for sequence-parallel runs (multi-GPU runs of the
+ * Sol-H3 runtime move Q, K, V as INT8 and the attention output as FP8, about
+ * half the inter-GPU bytes: ai-feiten.nl, "Videomodel MiniMax-H3 rendert
+ * sneller dan afspelen", "Waar de snelheidswinst vandaan komt").
+ *
+ * A row is the D bf16 channels of one (b, n, h).  Its fp32 scale is
+ * s = max|x| / L (L = 127 INT8, 448 e4m3); its codes are x / s (one fp32
+ * division each) rounded to nearest even, INT8 clamped to [-127, 127], e4m3
+ * saturating at +-448; an all-zero row has s = 0 and zero codes.  Dequantised
+ * values are bf16_rn(code * s) (one fp32 product).
+ *
+ * sol_quant_pack: x bf16 [B, N, H, D] -> codes (1 byte each) [G][B][Nc][Hc][D]
+ *   and scales fp32 [G][B][Nc][Hc], slice g holding what rank g receives:
+ *   SOL_SPLIT_HEADS  (token shard -> head shards): Hc = H/G, Nc = N, heads
+ *                    g*Hc .. g*Hc+Hc-1 (H % G == 0);
+ *   SOL_SPLIT_TOKENS (head shard -> token shards): Nc = N/G, Hc = H, tokens
+ *                    g*Nc .. g*Nc+Nc-1 (N % G == 0).
+ *   Slice g starts at row g * g_stride_rows of both buffers (0: B*Nc*Hc,
+ *   dense), so several tensors can share one exchange buffer.
+ * sol_dequant_unpack: codes / scales [G][B][Nc][Hc] (slice g from rank g, same
+ *   g_stride_rows rule) -> out bf16: SOL_SPLIT_HEADS concatenates the slices
+ *   along tokens, out [B, G*Nc, Hc, D] (token g*Nc + n); SOL_SPLIT_TOKENS
+ *   along heads, out [B, Nc, G*Hc, D] (head g*Hc + h).
+ * D in {64, 128}; x, out and codes 16-byte aligned, scales 4-byte aligned (device memory).
+ */
+typedef enum { SOL_CODE_INT8 = 0, SOL_CODE_E4M3 = 1 } sol_code;
+typedef enum { SOL_SPLIT_HEADS = 0, SOL_SPLIT_TOKENS = 1 } sol_split;
+sol_status sol_quant_pack(const void* x, int B, int N, int H, int D, int G, sol_split split, sol_code code,
+                          void* codes_out, float* scales_out, long long g_stride_rows, cudaStream_t stream);
+sol_status sol_dequant_unpack(const void* codes, const float* scales, int B, int Nc, int Hc, int D, int G,
+                              sol_split split, sol_code code, void* out, long long g_stride_rows,
+                              cudaStream_t stream);
+
+/*
  * sol_block_select_noalloc -- sol_block_select for callers that cannot
  * allocate device memory.  No counterpart on the pages: this is a convenience
  * of this library.

@@ -238,3 +238,28 @@ def test_select_ex_tile_checks(lib):
     assert f(FAKE, FAKE, OK_SHAPE, 64, 4, ctypes.byref(bad), FAKE, FAKE, None, None) == INVALID
     bad2 = Opts(2, 1.0, 0.0, None, Tile(1, 3, 8))      # does not divide the grid
     assert f(FAKE, FAKE, OK_SHAPE, 64, 4, ctypes.byref(bad2), FAKE, FAKE, None, None) == INVALID
+
+
+def test_quant_exchange_argument_checks(lib):
+    pack = lib.sol_quant_pack
+    pack.restype = ctypes.c_int
+    pack.argtypes = [ctypes.c_void_p] + [ctypes.c_int] * 7 + [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_longlong,
+                                                              ctypes.c_void_p]
+    # x, B, N, H, D, G, split, code, codes, scales, g_stride, stream
+    assert pack(None, 1, 96, 4, 128, 2, 0, 0, FAKE, FAKE, 0, None) == INVALID
+    assert pack(FAKE, 1, 96, 4, 128, 3, 0, 0, FAKE, FAKE, 0, None) == INVALID       # 4 heads over 3 ranks
+    assert pack(FAKE, 1, 96, 4, 128, 5, 1, 0, FAKE, FAKE, 0, None) == INVALID       # 96 tokens over 5 ranks
+    assert pack(FAKE, 1, 96, 4, 128, 2, 2, 0, FAKE, FAKE, 0, None) == INVALID       # unknown split
+    assert pack(FAKE, 1, 96, 4, 128, 2, 0, 7, FAKE, FAKE, 0, None) == INVALID       # unknown code
+    assert pack(FAKE, 1, 96, 4, 128, 2, 0, 0, FAKE, FAKE, 10, None) == INVALID      # slices overlap
+    assert pack(MISALIGNED, 1, 96, 4, 128, 2, 0, 0, FAKE, FAKE, 0, None) == INVALID
+    assert pack(FAKE, 1, 96, 4, 96, 2, 0, 0, FAKE, FAKE, 0, None) == UNSUPPORTED   # D = 96
+    unpack = lib.sol_dequant_unpack
+    unpack.restype = ctypes.c_int
+    unpack.argtypes = [ctypes.c_void_p, ctypes.c_void_p] + [ctypes.c_int] * 7 + [ctypes.c_void_p, ctypes.c_longlong,
+                                                                                 ctypes.c_void_p]
+    # codes, scales, B, Nc, Hc, D, G, split, code, out, g_stride, stream
+    assert unpack(FAKE, FAKE, 1, 48, 2, 128, 2, 0, 0, None, 0, None) == INVALID
+    assert unpack(FAKE, FAKE, 1, 48, 2, 128, 0, 0, 0, FAKE, 0, None) == INVALID     # G = 0
+    assert unpack(FAKE, FAKE, 1, 48, 2, 128, 2, 0, 0, FAKE, 95, None) == INVALID    # stride < 96 rows
+    assert unpack(FAKE, FAKE, 1, 48, 2, 32, 2, 0, 0, FAKE, 0, None) == UNSUPPORTED

@@ -76,3 +76,109 @@ def test_weak_scaling_value_counts_all_ranks():
     for world, ms in ((1, 30.0), (8, 31.0)):
         value = flops * world / (ms * 1e-3) / 1e12
         assert abs(value - world * flops / ms / 1e9) < 1e-6
+
+
+# ----------------------------------------------------------------------------- sequence-parallel exchange
+def _pack_np(x, plan, split, G, stride_rows, offset_rows, codes, scales):
+    """Host model of sol_quant_pack's documented layout (values copied, no quantisation):
+    x [B, Nx, Hx, D] -> slice g at row g * stride_rows + offset_rows + (b * Nc + n) * Hc + h."""
+    B, Nx, Hx, D = x.shape
+    for b in range(B):
+        for n in range(Nx):
+            for h in range(Hx):
+                if split == "heads":
+                    Hc, Nc = Hx // G, Nx
+                    g, nc, hc = h // Hc, n, h % Hc
+                else:
+                    Hc, Nc = Hx, Nx // G
+                    g, nc, hc = n // Nc, n % Nc, h
+                row = g * stride_rows + offset_rows + (b * Nc + nc) * Hc + hc
+                codes[row * D:(row + 1) * D] = x[b, n, h]
+                scales[row] = float(x[b, n, h, 0]) + 0.5
+
+
+def _seqpar_worker(rank, world, port, out_dir):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import torch.distributed as dist
+    from block_sparse_attention_sol_b200.seqpar import CollectiveTransport, ExchangePlan
+    dist.init_process_group("gloo", rank=rank, world_size=world, init_method=f"tcp://127.0.0.1:{port}")
+    B, N, H, D = 2, 12, 4, 8
+    plan = ExchangePlan(world, B, N, H, D)
+    Nl, Hg = plan.n_local, plan.h_local
+
+    def code(b, n, h, d):                      # identifies (batch, global token, global head, channel)
+        return (b * 101 + n * 7 + h * 13 + d) % 256
+
+    # this rank's token shard of Q, K, V (tensor t adds 50 * t)
+    shard = np.zeros((3, B, Nl, H, D), dtype=np.uint8)
+    for t in range(3):
+        for b in range(B):
+            for n in range(Nl):
+                for h in range(H):
+                    shard[t, b, n, h] = [(code(b, rank * Nl + n, h, d) + 50 * t) % 256 for d in range(D)]
+    send = np.zeros(plan.qkv_code_bytes, dtype=np.uint8)
+    send_s = np.zeros(plan.qkv_scale_count, dtype=np.float32)
+    for t in range(3):
+        _pack_np(shard[t], plan, "heads", world, plan.qkv_stride_rows, plan.qkv_offset_rows(t), send, send_s)
+    recv = torch.empty(plan.qkv_code_bytes, dtype=torch.uint8)
+    recv_s = torch.empty(plan.qkv_scale_count, dtype=torch.float32)
+    tr = CollectiveTransport()
+    tr.all_to_all(recv, torch.from_numpy(send))
+    tr.all_to_all(recv_s, torch.from_numpy(send_s))
+    recv, recv_s = recv.numpy(), recv_s.numpy()
+    # unpack as sol_dequant_unpack (split heads) documents: slice g -> tokens g * Nl ..
+    ok = True
+    for t in range(3):
+        for g in range(world):
+            for b in range(B):
+                for n in range(Nl):
+                    for h in range(Hg):
+                        row = g * plan.qkv_stride_rows + plan.qkv_offset_rows(t) + (b * Nl + n) * Hg + h
+                        n_glob, h_glob = g * Nl + n, rank * Hg + h
+                        want = [(code(b, n_glob, h_glob, d) + 50 * t) % 256 for d in range(D)]
+                        ok &= list(recv[row * D:(row + 1) * D]) == want
+                        ok &= recv_s[row] == float(want[0]) + 0.5
+    # the way back: this rank's head shard of O (all tokens) -> token shards, split tokens
+    o_h = np.zeros((B, N, Hg, D), dtype=np.uint8)
+    for b in range(B):
+        for n in range(N):
+            for h in range(Hg):
+                o_h[b, n, h] = [code(b, n, rank * Hg + h, d) for d in range(D)]
+    send_o = np.zeros(plan.o_code_bytes, dtype=np.uint8)
+    send_os = np.zeros(plan.o_scale_count, dtype=np.float32)
+    _pack_np(o_h, plan, "tokens", world, plan.rows, 0, send_o, send_os)
+    recv_o = torch.empty(plan.o_code_bytes, dtype=torch.uint8)
+    recv_os = torch.empty(plan.o_scale_count, dtype=torch.float32)
+    tr.all_to_all(recv_o, torch.from_numpy(send_o))
+    tr.all_to_all(recv_os, torch.from_numpy(send_os))
+    recv_o = recv_o.numpy()
+    for g in range(world):                      # slice g: heads g * Hg .. of this rank's tokens
+        for b in range(B):
+            for n in range(Nl):
+                for h in range(Hg):
+                    row = g * plan.rows + (b * Nl + n) * Hg + h
+                    want = [code(b, rank * Nl + n, g * Hg + h, d) for d in range(D)]
+                    ok &= list(recv_o[row * D:(row + 1) * D]) == want
+    with open(os.path.join(out_dir, f"seqpar_{rank}.txt"), "w") as f:
+        f.write("ok" if ok else "bad")
+    dist.destroy_process_group()
+
+
+@pytest.mark.timeout(300)
+def test_seqpar_exchange_layout_over_two_gloo_ranks(tmp_path):
+    port = _free_port()
+    mp.start_processes(_seqpar_worker, args=(2, port, str(tmp_path)), nprocs=2, join=True, start_method="spawn")
+    assert [open(tmp_path / f"seqpar_{r}.txt").read() for r in range(2)] == ["ok", "ok"]
+
+
+def test_exchange_plan_sizes_and_bytes():
+    from block_sparse_attention_sol_b200.seqpar import ExchangePlan
+    p = ExchangePlan(8, 1, 130560, 32, 128)
+    assert (p.n_local, p.h_local, p.rows) == (16320, 4, 65280)
+    assert p.qkv_code_bytes == 8 * 3 * 65280 * 128 and p.o_scale_count == 8 * 65280
+    # INT8 / FP8 codes plus one fp32 scale per 128 channels: 0.516 of the bf16 bytes
+    assert abs(p.wire_bytes() / p.bf16_wire_bytes() - 132 / 256) < 1e-12
+    with pytest.raises(ValueError):
+        ExchangePlan(3, 1, 130560, 32, 128)       # 32 heads do not split over 3 ranks
