@@ -5,8 +5,10 @@
 // "Videomodel MiniMax-H3 rendert sneller dan afspelen", section "Waar de
 // snelheidswinst vandaan komt").  Here a row is the D channels of one
 // (batch, token, head); each row gets one fp32 scale s = max|x| / L
-// (L = 127 for INT8, 448 for e4m3) and codes x / s rounded to nearest even
-// (INT8 clamped to +-127, e4m3 saturating), all decided in fp32.
+// (L = 127 for INT8, 448 for e4m3) and codes x * (L / max|x|) rounded to
+// nearest even (INT8 clamped to +-127, e4m3 saturating), all decided in fp32:
+// one division per row, one product per value (a division per value made the
+// kernel issue-bound on the XU pipe).
 //
 //   quant_pack:     bf16 rows [B, N, H, D] -> codes + scales packed by
 //                   destination rank g: [G][B][Nc][Hc][D] and [G][B][Nc][Hc].
@@ -49,13 +51,17 @@ __device__ __forceinline__ uint8_t encode(float q) {
   }
 }
 
+// Two codes (low byte first) of a 16-bit word as fp32, exactly.
 template <int CODE>
-__device__ __forceinline__ float decode(uint8_t c) {
+__device__ __forceinline__ float2 decode2(uint32_t w16) {
   if constexpr (CODE == kInt8) {
-    return static_cast<float>(static_cast<int8_t>(c));
+    // 2^23 + (c + 128) is exact in fp32: subtract 2^23 + 128 (no conversion instruction)
+    const uint32_t u = w16 ^ 0x8080u;
+    return make_float2(__uint_as_float(0x4B000000u | (u & 0xFFu)) - 8388736.0f,
+                       __uint_as_float(0x4B000000u | ((u >> 8) & 0xFFu)) - 8388736.0f);
   } else {
-    const __half_raw h = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(c), __NV_E4M3);
-    return __half2float(__half(h));
+    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w16), __NV_E4M3);
+    return __half22float2(__half2(h));
   }
 }
 
@@ -79,7 +85,9 @@ __global__ void __launch_bounds__(256) quant_pack_kernel(const __nv_bfloat16* __
   for (int e = 0; e < 8; ++e) a = fmaxf(a, fabsf(v[e]));
 #pragma unroll
   for (int o = L / 2; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(seg, a, o));
-  const float s = __fdiv_rn(a, CODE == kInt8 ? 127.0f : 448.0f);
+  const float levels = CODE == kInt8 ? 127.0f : 448.0f;
+  const float s = __fdiv_rn(a, levels);
+  const float rcp = __fdiv_rn(levels, a > 0.f ? a : 1.0f);
 
   const int h = static_cast<int>(row % H);
   const long long bn = row / H;
@@ -93,7 +101,7 @@ __global__ void __launch_bounds__(256) quant_pack_kernel(const __nv_bfloat16* __
   uint32_t w[2] = {0u, 0u};
   if (s > 0.f) {
 #pragma unroll
-    for (int e = 0; e < 8; ++e) w[e >> 2] |= static_cast<uint32_t>(encode<CODE>(__fdiv_rn(v[e], s))) << (8 * (e & 3));
+    for (int e = 0; e < 8; ++e) w[e >> 2] |= static_cast<uint32_t>(encode<CODE>(__fmul_rn(v[e], rcp))) << (8 * (e & 3));
   }
   __stcs(reinterpret_cast<uint2*>(codes + drow * D + li * 8), make_uint2(w[0], w[1]));
   if (li == 0) scales[drow] = s;
@@ -122,9 +130,8 @@ __global__ void __launch_bounds__(256) dequant_unpack_kernel(const uint8_t* __re
   uint32_t o[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const float lo = __fmul_rn(decode<CODE>(static_cast<uint8_t>(cw[i >> 1] >> (16 * (i & 1)))), s);
-    const float hi = __fmul_rn(decode<CODE>(static_cast<uint8_t>(cw[i >> 1] >> (16 * (i & 1) + 8))), s);
-    const __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+    const float2 c2 = decode2<CODE>((cw[i >> 1] >> (16 * (i & 1))) & 0xFFFFu);
+    const __nv_bfloat162 p = __floats2bfloat162_rn(__fmul_rn(c2.x, s), __fmul_rn(c2.y, s));
     o[i] = *reinterpret_cast<const uint32_t*>(&p);
   }
   long long orow;

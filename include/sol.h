@@ -264,9 +264,10 @@ sol_status sol_sparse_attn_fwd_tiled(const void* q, const void* k, const void* v
  * sneller dan afspelen", "Waar de snelheidswinst vandaan komt").
  *
  * A row is the D bf16 channels of one (b, n, h).  Its fp32 scale is
- * s = max|x| / L (L = 127 INT8, 448 e4m3); its codes are x / s (one fp32
- * division each) rounded to nearest even, INT8 clamped to [-127, 127], e4m3
- * saturating at +-448; an all-zero row has s = 0 and zero codes.  Dequantised
+ * s = max|x| / L (L = 127 INT8, 448 e4m3); its codes are x * r with
+ * r = L / max|x| (one fp32 division per row, one fp32 product per value)
+ * rounded to nearest even, INT8 clamped to [-127, 127], e4m3 saturating at
+ * +-448; an all-zero row has s = 0 and zero codes.  Dequantised
  * values are bf16_rn(code * s) (one fp32 product).
  *
  * sol_quant_pack: x bf16 [B, N, H, D] -> codes (1 byte each) [G][B][Nc][Hc][D]

@@ -12,10 +12,11 @@ details; the readings written out here are:
   - one scale per (token, head) row of D channels, symmetric, in fp32:
     s = max_d |x_d| / L with L = 127 (INT8) or 448 (FP8 e4m3, its largest
     finite value); a row of zeros gets s = 0 and all-zero codes;
-  - INT8 code = clamp(round_half_even(x / s), -127, 127); e4m3 code = x / s
-    rounded to the nearest e4m3 value (ties to even), saturating at +-448;
-    the quotient x / s is one IEEE fp32 division, and max, division and
-    rounding decide the code in fp32 exactly as written;
+  - the codes use the row's reciprocal scale r = L / max_d |x_d| (one IEEE
+    fp32 division per row): INT8 code = clamp(round_half_even(x * r), -127,
+    127); e4m3 code = x * r rounded to the nearest e4m3 value (ties to even),
+    saturating at +-448; x * r is one fp32 product, and max, division,
+    product and rounding decide the code in fp32 exactly as written;
   - dequantised value = bf16_round(fp32(code * s)).
   - sequence-parallel layout: G ranks; rank r owns tokens [r N/G, (r+1) N/G)
     of all heads before the attention and heads [r H/G, (r+1) H/G) of all
@@ -62,8 +63,9 @@ def quantize_rows(x, kind: str):
     levels = np.float32(INT8_LEVELS if kind == "int8" else E4M3_MAX)
     amax = np.max(np.abs(x32), axis=-1)
     s = (amax / levels).astype(np.float32)                       # one fp32 division
-    safe = np.where(s > 0, s, np.float32(1.0)).astype(np.float32)
-    quo = (x32 / safe[..., None]).astype(np.float32)             # one fp32 division per value
+    safe = np.where(amax > 0, amax, np.float32(1.0)).astype(np.float32)
+    recip = (levels / safe).astype(np.float32)                   # one fp32 division per row
+    quo = (x32 * recip[..., None]).astype(np.float32)            # one fp32 product per value
     if kind == "int8":
         codes = np.clip(np.rint(quo.astype(np.float64)), -127.0, 127.0)
     elif kind == "e4m3":

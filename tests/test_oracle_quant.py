@@ -37,7 +37,8 @@ def test_int8_codes_brute_force():
         if s[r] == 0:
             assert (codes[r] == 0).all()
             continue
-        quo = (x[r] / s[r]).astype(np.float32).astype(np.float64)
+        recip = np.float32(127.0) / np.abs(x[r]).max()
+        quo = (x[r] * recip).astype(np.float32).astype(np.float64)
         for d in range(x.shape[1]):
             dist = np.abs(levels - quo[d])
             best = levels[dist == dist.min()]
