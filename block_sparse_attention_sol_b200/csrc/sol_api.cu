@@ -455,6 +455,19 @@ sol_status sol_block_select_pooled_ex(const float* qbar, const float* kbar, sol_
   return launch_score_topk(di, s.D, plan, stream, qbar, kbar, a);
 }
 
+}  // extern "C"
+
+namespace {
+// Threads per CTA of the exchange kernels: D / 8 lanes for each of `rows` rows, at most 1024.
+int quant_block(int rows, int D) { return std::min(rows * (D / 8), 1024); }
+// CTAs of the exchange kernels: two resident waves (2048 threads per SM), the CTAs loop over tokens.
+long long quant_grid(const DeviceInfo* di, int threads) {
+  return 2ll * di->sm_count * std::max(1, 2048 / threads);
+}
+}  // namespace
+
+extern "C" {
+
 sol_status sol_quant_pack(const void* x, int B, int N, int H, int D, int G, sol_split split, sol_code code,
                           void* codes_out, float* scales_out, long long g_stride_rows, cudaStream_t stream) {
   if (!x || !codes_out || !scales_out) return SOL_ERR_INVALID_ARG;
@@ -467,25 +480,26 @@ sol_status sol_quant_pack(const void* x, int B, int N, int H, int D, int G, sol_
   if (g_stride_rows == 0) g_stride_rows = per_g;
   if (g_stride_rows < per_g) return SOL_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return SOL_ERR_UNSUPPORTED;
-  const long long threads = static_cast<long long>(B) * N * H * (D / 8);
-  const long long grid = (threads + 255) / 256;
-  if (grid > 0x7fffffffll) return SOL_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * N * H >= 0x7fffffffll) return SOL_ERR_UNSUPPORTED;
   const auto* xb = static_cast<const __nv_bfloat16*>(x);
   auto* cb = static_cast<uint8_t*>(codes_out);
-  const dim3 g(static_cast<unsigned>(grid));
+  const int threads = quant_block(H, D);
+  DeviceInfo* di = nullptr;
+  if (sol_status st = device_info(&di)) return st;
+  const dim3 g(static_cast<unsigned>(std::min<long long>(static_cast<long long>(B) * N, quant_grid(di, threads))));
   if (D == 128) {
     if (code == SOL_CODE_INT8)
-      sol::quant::quant_pack_kernel<128, sol::quant::kInt8><<<g, 256, 0, stream>>>(xb, cb, scales_out, B, N, H, G, split,
+      sol::quant::quant_pack_kernel<128, sol::quant::kInt8><<<g, threads, 0, stream>>>(xb, cb, scales_out, B, N, H, G, split,
                                                                                    g_stride_rows);
     else
-      sol::quant::quant_pack_kernel<128, sol::quant::kE4M3><<<g, 256, 0, stream>>>(xb, cb, scales_out, B, N, H, G, split,
+      sol::quant::quant_pack_kernel<128, sol::quant::kE4M3><<<g, threads, 0, stream>>>(xb, cb, scales_out, B, N, H, G, split,
                                                                                    g_stride_rows);
   } else {
     if (code == SOL_CODE_INT8)
-      sol::quant::quant_pack_kernel<64, sol::quant::kInt8><<<g, 256, 0, stream>>>(xb, cb, scales_out, B, N, H, G, split,
+      sol::quant::quant_pack_kernel<64, sol::quant::kInt8><<<g, threads, 0, stream>>>(xb, cb, scales_out, B, N, H, G, split,
                                                                                   g_stride_rows);
     else
-      sol::quant::quant_pack_kernel<64, sol::quant::kE4M3><<<g, 256, 0, stream>>>(xb, cb, scales_out, B, N, H, G, split,
+      sol::quant::quant_pack_kernel<64, sol::quant::kE4M3><<<g, threads, 0, stream>>>(xb, cb, scales_out, B, N, H, G, split,
                                                                                   g_stride_rows);
   }
   return launch_status();
@@ -502,25 +516,26 @@ sol_status sol_dequant_unpack(const void* codes, const float* scales, int B, int
   if (g_stride_rows == 0) g_stride_rows = per_g;
   if (g_stride_rows < per_g) return SOL_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return SOL_ERR_UNSUPPORTED;
-  const long long threads = G * per_g * (D / 8);
-  const long long grid = (threads + 255) / 256;
-  if (grid > 0x7fffffffll) return SOL_ERR_UNSUPPORTED;
+  if (G * per_g >= 0x7fffffffll) return SOL_ERR_UNSUPPORTED;
   const auto* cb = static_cast<const uint8_t*>(codes);
   auto* ob = static_cast<__nv_bfloat16*>(out);
-  const dim3 g(static_cast<unsigned>(grid));
+  const int threads = quant_block(Hc, D);
+  DeviceInfo* di = nullptr;
+  if (sol_status st = device_info(&di)) return st;
+  const dim3 g(static_cast<unsigned>(std::min<long long>(static_cast<long long>(G) * B * Nc, quant_grid(di, threads))));
   if (D == 128) {
     if (code == SOL_CODE_INT8)
-      sol::quant::dequant_unpack_kernel<128, sol::quant::kInt8><<<g, 256, 0, stream>>>(cb, scales, ob, B, Nc, Hc, G,
+      sol::quant::dequant_unpack_kernel<128, sol::quant::kInt8><<<g, threads, 0, stream>>>(cb, scales, ob, B, Nc, Hc, G,
                                                                                        split, g_stride_rows);
     else
-      sol::quant::dequant_unpack_kernel<128, sol::quant::kE4M3><<<g, 256, 0, stream>>>(cb, scales, ob, B, Nc, Hc, G,
+      sol::quant::dequant_unpack_kernel<128, sol::quant::kE4M3><<<g, threads, 0, stream>>>(cb, scales, ob, B, Nc, Hc, G,
                                                                                        split, g_stride_rows);
   } else {
     if (code == SOL_CODE_INT8)
-      sol::quant::dequant_unpack_kernel<64, sol::quant::kInt8><<<g, 256, 0, stream>>>(cb, scales, ob, B, Nc, Hc, G,
+      sol::quant::dequant_unpack_kernel<64, sol::quant::kInt8><<<g, threads, 0, stream>>>(cb, scales, ob, B, Nc, Hc, G,
                                                                                       split, g_stride_rows);
     else
-      sol::quant::dequant_unpack_kernel<64, sol::quant::kE4M3><<<g, 256, 0, stream>>>(cb, scales, ob, B, Nc, Hc, G,
+      sol::quant::dequant_unpack_kernel<64, sol::quant::kE4M3><<<g, threads, 0, stream>>>(cb, scales, ob, B, Nc, Hc, G,
                                                                                       split, g_stride_rows);
   }
   return launch_status();
