@@ -458,9 +458,9 @@ sol_status sol_block_select_pooled_ex(const float* qbar, const float* kbar, sol_
 }  // extern "C"
 
 namespace {
-// Threads per CTA of the exchange kernels: D / 8 lanes per row, at most 512
+// Threads per CTA of the exchange kernels: D / 16 lanes per row, at most 512
 // (each thread takes two rows per pass, so half the rows' lanes suffice)
-int quant_block(int rows, int D) { return std::min(((rows + 1) / 2) * (D / 8), 512); }
+int quant_block(int rows, int D) { return std::min(((rows + 1) / 2) * (D / 16), 512); }
 // CTAs of the exchange kernels: two resident waves (2048 threads per SM), the CTAs loop over tokens.
 long long quant_grid(const DeviceInfo* di, int threads) {
   return 2ll * di->sm_count * std::max(1, 2048 / threads);
