@@ -53,15 +53,16 @@ __device__ __forceinline__ uint4 encode16(const uint32_t (&w)[8], unsigned seg, 
   if constexpr (CODE == kInt8) {
     // |x * rcp| <= 127 (1 + 2^-23): no clamp needed.  q + 1.5 * 2^23 rounds q to
     // the nearest (even) integer, held in the sum's low mantissa bits: its low
-    // byte is the two's complement code.
-    const uint64_t magic2 = f2_pack(12582912.0f, 12582912.0f);
+    // byte is the two's complement code.  The product must be rounded before the
+    // add (a fused multiply-add rounds ties such as 63.5 the other way), so the
+    // add is a scalar __fadd_rn, which is never contracted.
     uint32_t b[16];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const uint64_t y = f2_add(f2_mul(f2_pack(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u)),
-                                       rcp2), magic2);
-      b[2 * i] = static_cast<uint32_t>(y);
-      b[2 * i + 1] = static_cast<uint32_t>(y >> 32);
+      float lo, hi;
+      f2_unpack(f2_mul(f2_pack(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u)), rcp2), lo, hi);
+      b[2 * i] = __float_as_uint(__fadd_rn(lo, 12582912.0f));
+      b[2 * i + 1] = __float_as_uint(__fadd_rn(hi, 12582912.0f));
     }
 #pragma unroll
     for (int k = 0; k < 4; ++k)
