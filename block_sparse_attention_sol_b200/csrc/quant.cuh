@@ -178,7 +178,10 @@ __global__ void __launch_bounds__(512) quant_pack_kernel(const __nv_bfloat16* __
 }
 
 // A CTA handles a contiguous run of received row groups (g, b, nc); thread t
-// handles channels 16 (t % L) .. +15 of heads hc = t / L + k S, two per pass.
+// handles channels 16 (t % L) .. +15 of heads hc = t / L + k S, kUnpackRows per
+// pass with all their loads issued first (the kernel is latency-bound otherwise).
+constexpr int kUnpackRows = 4;
+
 template <int D, int CODE>
 __global__ void __launch_bounds__(512) dequant_unpack_kernel(const uint8_t* __restrict__ codes,
                                                              const float* __restrict__ scales,
@@ -198,19 +201,24 @@ __global__ void __launch_bounds__(512) dequant_unpack_kernel(const uint8_t* __re
     long long obase;   // output row of hc = 0
     if (split == kSplitHeads) obase = (static_cast<long long>(b) * G * Nc + static_cast<long long>(g) * Nc + nc) * Hc;
     else obase = (static_cast<long long>(b) * Nc + nc) * (static_cast<long long>(G) * Hc) + static_cast<long long>(g) * Hc;
-    for (int hc = threadIdx.x / L; hc < Hc; hc += 2 * S) {
-      const int hc2 = hc + S;
-      const bool two = hc2 < Hc;
-      const uint4 c1 = __ldcs(reinterpret_cast<const uint4*>(codes + (rbase + hc) * D + li * 16));
-      const uint4 c2 = two ? __ldcs(reinterpret_cast<const uint4*>(codes + (rbase + hc2) * D + li * 16)) : c1;
-      const float s1 = __ldg(scales + rbase + hc);
-      const float s2 = two ? __ldg(scales + rbase + hc2) : s1;
+    for (int hc = threadIdx.x / L; hc < Hc; hc += kUnpackRows * S) {
+      uint4 c[kUnpackRows];
+      float sc[kUnpackRows];
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        if (u == 1 && !two) break;
+      for (int u = 0; u < kUnpackRows; ++u) {
+        const int hu = hc + u * S;
+        if (hu < Hc) {
+          c[u] = __ldcs(reinterpret_cast<const uint4*>(codes + (rbase + hu) * D + li * 16));
+          sc[u] = __ldg(scales + rbase + hu);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kUnpackRows; ++u) {
+        const int hu = hc + u * S;
+        if (hu >= Hc) break;
         uint32_t o[8];
-        decode16<CODE>(u ? c2 : c1, u ? s2 : s1, o);
-        uint4* dst = reinterpret_cast<uint4*>(out + (obase + (u ? hc2 : hc)) * D + li * 16);
+        decode16<CODE>(c[u], sc[u], o);
+        uint4* dst = reinterpret_cast<uint4*>(out + (obase + hu) * D + li * 16);
         __stcs(dst, make_uint4(o[0], o[1], o[2], o[3]));
         __stcs(dst + 1, make_uint4(o[4], o[5], o[6], o[7]));
       }

@@ -520,7 +520,7 @@ sol_status sol_dequant_unpack(const void* codes, const float* scales, int B, int
   if (G * per_g >= 0x7fffffffll) return SOL_ERR_UNSUPPORTED;
   const auto* cb = static_cast<const uint8_t*>(codes);
   auto* ob = static_cast<__nv_bfloat16*>(out);
-  const int threads = quant_block(Hc, D);
+  const int threads = std::min(((Hc + sol::quant::kUnpackRows - 1) / sol::quant::kUnpackRows) * (D / 16), 512);
   DeviceInfo* di = nullptr;
   if (sol_status st = device_info(&di)) return st;
   const dim3 g(static_cast<unsigned>(std::min<long long>(static_cast<long long>(G) * B * Nc, quant_grid(di, threads))));
