@@ -179,8 +179,8 @@ __global__ void __launch_bounds__(512) quant_pack_kernel(const __nv_bfloat16* __
 
 // A CTA handles a contiguous run of received row groups (g, b, nc); thread t
 // handles channels 16 (t % L) .. +15 of heads hc = t / L + k S, kUnpackRows per
-// pass with all their loads issued first (the kernel is latency-bound otherwise).
-constexpr int kUnpackRows = 4;
+// pass with all their loads issued first (four cost occupancy and ran slower).
+constexpr int kUnpackRows = 2;
 
 template <int D, int CODE>
 __global__ void __launch_bounds__(512) dequant_unpack_kernel(const uint8_t* __restrict__ codes,
