@@ -86,3 +86,51 @@ def quant_roundtrip(x, kind: str) -> np.ndarray:
     """The values a tensor [..., D] arrives with after quantisation and dequantisation."""
     codes, s = quantize_rows(x, kind)
     return dequantize_rows(codes, s)
+
+
+# ----------------------------------------------------------------------------- FP8 attention inputs
+# Readings for the FP8 (e4m3) variant of the attention (the pages say only that
+# the runtime uses FP8; the formats are this library's): Q and K rows are
+# quantised like the exchange rows above (one scale per (token, head) row);
+# V gets one scale per (batch, head), s_v = max |v| over all its tokens and
+# channels / 448, codes v * (448 / max |v|) rounded to nearest e4m3.  The
+# attention is then the exact softmax attention of the dequantised values
+# (code * scale, in fp64 here); the kernel's further rounding of P to e4m3 is
+# an approximation that the tests bound.
+__all__ += ["quantize_heads_e4m3", "fp8_attention_inputs", "VT_KEY_ORDER"]
+
+# V is stored transposed, [B, H, D, N], with the keys of every aligned group of
+# 16 in this order (position j of the group holds key VT_KEY_ORDER[j]).
+VT_KEY_ORDER = (0, 1, 8, 9, 2, 3, 10, 11, 4, 5, 12, 13, 6, 7, 14, 15)
+
+
+def quantize_heads_e4m3(v):
+    """v [B, N, H, D] -> (codes float64 [B, N, H, D], scales float32 [B, H]), one scale per (b, h)."""
+    v32 = np.asarray(v, dtype=np.float32)
+    amax = np.max(np.abs(v32), axis=(1, 3))                       # [B, H]
+    s = (amax / np.float32(E4M3_MAX)).astype(np.float32)
+    safe = np.where(amax > 0, amax, np.float32(1.0)).astype(np.float32)
+    recip = (np.float32(E4M3_MAX) / safe).astype(np.float32)
+    quo = (v32 * recip[:, None, :, None]).astype(np.float32)
+    codes = e4m3_round(quo.astype(np.float64))
+    codes = np.where(s[:, None, :, None] > 0, codes, 0.0)
+    return codes, s
+
+
+def fp8_attention_inputs(q, k, v):
+    """Codes, scales and the dequantised (exact, fp64) Q, K, V of the FP8 attention.
+
+    Returns dict with q_codes, q_scales [B, H, N], k_codes, k_scales [B, H, N],
+    v_codes [B, N, H, D], v_scales [B, H], and q_deq, k_deq, v_deq (float64
+    [B, N, H, D], code * scale without further rounding)."""
+    qc, qs = quantize_rows(q, "e4m3")                               # scales [B, N, H]
+    kc, ks = quantize_rows(k, "e4m3")
+    vc, vs = quantize_heads_e4m3(v)
+    return {
+        "q_codes": qc, "q_scales": np.ascontiguousarray(np.swapaxes(qs, 1, 2)),
+        "k_codes": kc, "k_scales": np.ascontiguousarray(np.swapaxes(ks, 1, 2)),
+        "v_codes": vc, "v_scales": vs,
+        "q_deq": qc * qs.astype(np.float64)[..., None],
+        "k_deq": kc * ks.astype(np.float64)[..., None],
+        "v_deq": vc * vs.astype(np.float64)[:, None, :, None],
+    }

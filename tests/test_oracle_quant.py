@@ -71,3 +71,34 @@ def test_roundtrip_error_bounds(kind, rel):
     else:
         bound = rel * np.abs(x) + 2.0 ** -10 * amax / 448.0 + 2.0 ** -8 * np.abs(y)
     assert (np.abs(y - x) <= bound + 1e-12).all()
+
+
+def test_head_scales_fp8_inputs():
+    rng = np.random.default_rng(14)
+    v = rng.standard_normal((2, 48, 3, 16)).astype(np.float32)
+    v[1, :, 2] = 0.0                                          # an all-zero head
+    codes, s = orc.quantize_heads_e4m3(v)
+    for b in range(2):
+        for h in range(3):
+            a = np.abs(v[b, :, h]).max()
+            assert s[b, h] == np.float32(a / np.float32(448.0))
+            if a == 0:
+                assert (codes[b, :, h] == 0).all()
+                continue
+            # codes are the e4m3 values nearest to v * (448 / amax), checked against torch's cast
+            quo = (v[b, :, h] * (np.float32(448.0) / np.float32(a))).astype(np.float32)
+            want = torch.from_numpy(np.clip(quo, -448, 448)).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+            assert np.array_equal(codes[b, :, h], want)
+            assert np.abs(codes[b, :, h]).max() == 448.0
+    d = orc.fp8_attention_inputs(v, v, v)
+    assert d["q_scales"].shape == (2, 3, 48) and d["v_scales"].shape == (2, 3)
+    assert np.allclose(d["v_deq"], v, rtol=2.0 ** -4, atol=2.0 ** -10 * np.abs(v).max() / 448 * 2)
+
+
+def test_vt_key_order_is_a_permutation_of_each_16_group():
+    order = orc.VT_KEY_ORDER
+    assert sorted(order) == list(range(16))
+    # position 4 c + e of a group (TMEM column c, byte e) holds key 2 c + (e & 1) + 8 (e >> 1)
+    for pos in range(16):
+        c, e = pos // 4, pos % 4
+        assert order[pos] == 2 * c + (e & 1) + 8 * (e >> 1)
