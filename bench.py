@@ -303,6 +303,34 @@ def run_ours(args, wl, world, rank, local):
     alt_ms = {name: sum(e[i].elapsed_time(e[i + 1]) for e in alt_evs) / alt_steps
               for i, name in enumerate(("prologue", "select", "attention"))}
 
+    # FP8 (e4m3) variant of the attention on the same prologue outputs and selection,
+    # for comparison (not part of `value`: reduced precision).  Its peak is the
+    # measured bf16 rate x 2, the nominal e4m3 / bf16 ratio of the tensor cores.
+    fp8 = None
+    if not args.no_fp8:
+        fin = sol.sol_quant_attn_fp8(q, k, d["v"], wl.grid)
+        o8 = torch.empty_like(o)
+        lse8 = torch.empty_like(lse)
+        fp8_steps = min(args.steps, 10)
+        e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        sol.sol_sparse_attn_fwd_fp8(fin, idx, wl.grid, wl.block, o=o8, lse=lse8)
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for _ in range(fp8_steps):
+            sol.sol_quant_attn_fp8(q, k, d["v"], wl.grid, out=fin)
+        e1.record(stream)
+        for _ in range(fp8_steps):
+            sol.sol_sparse_attn_fwd_fp8(fin, idx, wl.grid, wl.block, o=o8, lse=lse8)
+        e2.record(stream)
+        torch.cuda.synchronize(dev)
+        qms = e0.elapsed_time(e1) / fp8_steps
+        ams = e1.elapsed_time(e2) / fp8_steps
+        io_b = wl.B * wl.N * wl.H * wl.D * 2
+        # read q, k once and v twice (its per-head max, then its codes); write three
+        # e4m3 code tensors and the q, k row scales
+        qbytes = 4 * io_b + 3 * io_b // 2 + 2 * 4 * wl.B * wl.H * wl.N
+        fp8 = {"quantise_ms": qms, "quantise_GB/s": qbytes / qms / 1e6,
+               "attention_ms": ams, "attention_TFLOP/s": wl.selected_flops(topk) / ams / 1e9}
     # End to end through host buffers, the way a caller streams clips: the pipeline
     # copies each step's raw Q, K, V in from pinned host memory, runs the fused chain
     # and copies O and LSE back, with the next step's inputs crossing PCIe while the
@@ -366,6 +394,13 @@ def run_ours(args, wl, world, rank, local):
     pooled_bytes = 2 * wl.B * wl.H * wl.nb * wl.D * 4
     score_flops = 2 * wl.B * wl.H * wl.nb * wl.nb * wl.D
 
+    if fp8 is not None:
+        fp8["peak_tflops_e4m3"] = 2 * peaks["bf16_tflops"]
+        fp8["frac_e4m3_burst"] = fp8["attention_TFLOP/s"] / fp8["peak_tflops_e4m3"]
+        fp8["frac_e4m3_sustained"] = fp8["attention_TFLOP/s"] / (2 * peak)
+        fp8["quantise_frac_hbm"] = fp8["quantise_GB/s"] / peaks["hbm_gbs"]
+        fp8["kernel"] = "sol::attnfp8::sparse_attn_fp8_kernel"
+
     def stages(st, fused):
         """Per-stage rates.  Algorithmic bytes: prologue reads q_raw, k_raw and writes
         q, k (+ the block means when fused); the split selection reads q, k and writes
@@ -414,6 +449,7 @@ def run_ours(args, wl, world, rank, local):
             "ms_per_step": e2e_ms, "api": "block_sparse_attention_sol_b200.pipeline.HostChainPipeline",
             "overlap": "double-buffered over clips: step i+1's inputs cross PCIe while step i computes",
             "serial_ms_per_step": e2e_serial_ms},
+        "fp8_attention": fp8,
         "gpu_launches": (3 if args.chain == "fused" else 4) * args.steps,
         "clocks": clocks,
     }
@@ -524,6 +560,7 @@ def main():
     ap.add_argument("--ref-units", type=int, default=24)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="profiling runs: skip the end-to-end runs")
+    ap.add_argument("--no-fp8", action="store_true", help="skip the FP8 attention comparison")
     ap.add_argument("--chain", choices=("fused", "split"), default="fused",
                     help="fused: prologue emits the block means (3 launches per step); split: the selection "
                          "pools q and k itself (4 launches)")

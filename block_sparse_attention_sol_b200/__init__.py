@@ -17,6 +17,8 @@ Functions (same names as the C ABI):
     sol_sparse_attn_fwd_tiled(q, k, v, idx, grid, tile, counts=None, ...) -> (o, lse)
     sol_quant_pack(x, G, split, code, codes_out, scales_out, ...)  (exchange buffers)
     sol_dequant_unpack(codes, scales, B, Nc, Hc, D, G, split, code, out, ...)
+    sol_quant_attn_fp8(q, k, v, grid) -> dict of e4m3 codes and scales
+    sol_sparse_attn_fwd_fp8(fp8_inputs, idx, grid, block, counts=None, ...) -> (o, lse)
     sol_check_device_status(stream=None)
     sol_selftest_wait_timeout(limit_us, stream=None)
     sol_block_select_workspace_bytes(shape, block)
@@ -32,7 +34,7 @@ __all__ = [
     "SolError", "SolShape", "LIB_PATH", "lib",
     "sol_qk_prologue", "sol_block_select", "sol_block_select_workspace_bytes", "sol_sparse_attn_fwd",
     "sol_qk_prologue_pool", "sol_block_select_pooled", "sol_block_select_pooled_ex", "sol_sparse_attn_fwd_counts",
-    "SolSelectOpts", "SolTile", "sol_quant_pack", "sol_dequant_unpack",
+    "SolSelectOpts", "SolTile", "sol_quant_pack", "sol_dequant_unpack", "sol_quant_attn_fp8", "sol_sparse_attn_fwd_fp8",
     "SOL_CODE_INT8", "SOL_CODE_E4M3", "SOL_SPLIT_HEADS", "SOL_SPLIT_TOKENS", "sol_qk_prologue_pool_tiled", "sol_sparse_attn_fwd_tiled", "SOL_SELECT_FORCE_DIAGONAL", "SOL_SELECT_FORCE_FIRST_FRAME", "SOL_SELECT_TOP_P",
     "sol_check_device_status", "sol_selftest_wait_timeout", "sol_status_string", "sol_attention_chain",
     "SOL_OK", "SOL_ERR_INVALID_ARG", "SOL_ERR_UNSUPPORTED", "SOL_ERR_CUDA", "SOL_ERR_TIMEOUT",
@@ -97,6 +99,12 @@ lib.sol_quant_pack.restype = _I
 lib.sol_quant_pack.argtypes = [_P, _I, _I, _I, _I, _I, _I, _I, _P, _P, ctypes.c_longlong, _P]
 lib.sol_dequant_unpack.restype = _I
 lib.sol_dequant_unpack.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _I, _P, ctypes.c_longlong, _P]
+lib.sol_quant_attn_fp8_workspace_bytes.restype = _SZ
+lib.sol_quant_attn_fp8_workspace_bytes.argtypes = [SolShape]
+lib.sol_quant_attn_fp8.restype = _I
+lib.sol_quant_attn_fp8.argtypes = [_P, _P, _P, SolShape, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
+lib.sol_sparse_attn_fwd_fp8.restype = _I
+lib.sol_sparse_attn_fwd_fp8.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, SolShape, _I, _I, _F, _P, _P, _P]
 lib.sol_sparse_attn_fwd.restype = _I
 lib.sol_sparse_attn_fwd.argtypes = [_P, _P, _P, _P, SolShape, _I, _I, _F, _I, _P, _P, _P]
 lib.sol_check_device_status.restype = _I
@@ -358,6 +366,52 @@ def sol_dequant_unpack(codes, scales, B, Nc, Hc, D, G, split, code, out, g_strid
     st = lib.sol_dequant_unpack(codes.data_ptr(), scales.data_ptr(), int(B), int(Nc), int(Hc), int(D), int(G), int(split),
                                 int(code), out.data_ptr(), int(g_stride_rows), _stream_handle(stream))
     _check(st, "sol_dequant_unpack")
+
+
+def sol_quant_attn_fp8(q, k, v, grid, out=None, stream=None):
+    """e4m3 codes and scales of bf16 q, k, v [B, N, H, D] for sol_sparse_attn_fwd_fp8 (layouts in include/sol.h).
+    Returns a dict: q8, q_scale [B, H, N], k8, k_scale, vt8 [B, H, D, N], v_scale [B, H]."""
+    _cuda(q, "q"), _cuda(k, "k"), _cuda(v, "v")
+    if q.dtype != torch.bfloat16 or k.dtype != torch.bfloat16 or v.dtype != torch.bfloat16:
+        raise TypeError("q, k, v must be bf16")
+    s = _shape(q, grid)
+    dev = q.device
+    if out is None:
+        out = {"q8": torch.empty(q.shape, dtype=torch.uint8, device=dev),
+               "k8": torch.empty(k.shape, dtype=torch.uint8, device=dev),
+               "vt8": torch.empty((s.B, s.H, s.D, s.N), dtype=torch.uint8, device=dev),
+               "q_scale": torch.empty((s.B, s.H, s.N), dtype=torch.float32, device=dev),
+               "k_scale": torch.empty((s.B, s.H, s.N), dtype=torch.float32, device=dev),
+               "v_scale": torch.empty((s.B, s.H), dtype=torch.float32, device=dev)}
+        ws = max(int(lib.sol_quant_attn_fp8_workspace_bytes(s)), 16)
+        out["workspace"] = torch.empty(ws, dtype=torch.uint8, device=dev)
+    st = lib.sol_quant_attn_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), s, out["q8"].data_ptr(),
+                                out["q_scale"].data_ptr(), out["k8"].data_ptr(), out["k_scale"].data_ptr(),
+                                out["vt8"].data_ptr(), out["v_scale"].data_ptr(), out["workspace"].data_ptr(),
+                                out["workspace"].numel(), _stream_handle(stream))
+    _check(st, "sol_quant_attn_fp8")
+    return out
+
+
+def sol_sparse_attn_fwd_fp8(fp8, idx, grid, block, counts=None, softmax_scale=0.0, o=None, lse=None, stream=None):
+    """Attention on e4m3 operands (fp8: the dict of sol_quant_attn_fp8, or the same keys).  Returns (o bf16, lse)."""
+    for n in ("q8", "k8", "vt8", "q_scale", "k_scale", "v_scale"):
+        _cuda(fp8[n], n)
+    _cuda(idx, "idx")
+    if idx.dtype != torch.int32 or (counts is not None and counts.dtype != torch.int32):
+        raise TypeError("idx and counts must be int32")
+    q8 = fp8["q8"]
+    B, N, H, D = q8.shape
+    s = SolShape(B, N, H, D, int(grid[0]), int(grid[1]), int(grid[2]))
+    o = torch.empty((B, N, H, D), dtype=torch.bfloat16, device=q8.device) if o is None else _cuda(o, "o")
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q8.device) if lse is None else _cuda(lse, "lse")
+    st = lib.sol_sparse_attn_fwd_fp8(q8.data_ptr(), fp8["q_scale"].data_ptr(), fp8["k8"].data_ptr(),
+                                     fp8["k_scale"].data_ptr(), fp8["vt8"].data_ptr(), fp8["v_scale"].data_ptr(),
+                                     idx.data_ptr(), _cuda(counts, "counts").data_ptr() if counts is not None else None,
+                                     s, int(block), int(idx.shape[-1]), float(softmax_scale), o.data_ptr(),
+                                     lse.data_ptr(), _stream_handle(stream))
+    _check(st, "sol_sparse_attn_fwd_fp8")
+    return o, lse
 
 
 def sol_check_device_status(stream=None) -> int:

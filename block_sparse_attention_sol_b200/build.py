@@ -42,7 +42,7 @@ def _stale() -> bool:
 
 
 # Kernels whose spilling would silently cost performance: the build refuses them.
-NO_SPILL_KERNELS = ("sparse_attn_fwd_kernel",)
+NO_SPILL_KERNELS = ("sparse_attn_fwd_kernel", "sparse_attn_fp8_kernel")
 
 
 # Kernels that split their registers between warpgroups with setmaxnreg: the split

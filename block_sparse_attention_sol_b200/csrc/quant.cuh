@@ -230,5 +230,136 @@ __global__ void __launch_bounds__(512) dequant_unpack_kernel(const uint8_t* __re
   }
 }
 
+// ------------------------------------------------------------------ FP8 attention inputs
+// Q or K rows -> e4m3 codes [B, N, H, D] and per-row scales laid out [B, H, N]
+// (the attention kernel reads a block's 128 key scales contiguously).  Same
+// arithmetic as quant_pack_kernel with G = 1.
+template <int D>
+__global__ void __launch_bounds__(512) quant_rows_e4m3_kernel(const __nv_bfloat16* __restrict__ x,
+                                                              uint8_t* __restrict__ codes,
+                                                              float* __restrict__ scales, int B, int N, int H) {
+  constexpr int L = D / 16;
+  const int li = threadIdx.x % L;
+  const int S = blockDim.x / L;
+  const unsigned lane = threadIdx.x & 31u;
+  const unsigned seg = (((1u << L) - 1u) << (lane & ~static_cast<unsigned>(L - 1)));
+  const int total = B * N;
+  const int chunk = (total + gridDim.x - 1) / gridDim.x;
+  const int t0 = blockIdx.x * chunk, t1 = min(total, t0 + chunk);
+  if (t0 >= t1) return;
+  int b = t0 / N, n = t0 - b * N;
+  for (int tok = t0; tok < t1; ++tok) {
+    const long long rowbase = static_cast<long long>(tok) * H;
+    for (int h = threadIdx.x / L; h < H; h += S) {
+      const __nv_bfloat16* src = x + (rowbase + h) * D + li * 16;
+      const uint4 r0 = __ldcs(reinterpret_cast<const uint4*>(src));
+      const uint4 r1 = __ldcs(reinterpret_cast<const uint4*>(src + 8));
+      const uint32_t w[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+      float sc;
+      const uint4 cw = encode16<L, kE4M3>(w, seg, &sc);
+      __stcs(reinterpret_cast<uint4*>(codes + (rowbase + h) * D + li * 16), cw);
+      if (li == 0) scales[(static_cast<long long>(b) * H + h) * N + n] = sc;
+    }
+    if (++n == N) { n = 0; ++b; }
+  }
+}
+
+// max |v| per (b, h) over all tokens and channels, as the bits of a
+// non-negative float (ordered like unsigned integers), into amax_bits [B * H]
+// (zeroed by the host).  A CTA walks a run of tokens and keeps one running max
+// per (thread, head); it flushes with atomicMax when the batch index changes.
+template <int D>
+__global__ void __launch_bounds__(256) head_amax_kernel(const __nv_bfloat16* __restrict__ v,
+                                                        unsigned* __restrict__ amax_bits, int B, int N, int H) {
+  constexpr int L = D / 16;
+  const int li = threadIdx.x % L;
+  const int S = blockDim.x / L;
+  const unsigned lane = threadIdx.x & 31u;
+  const unsigned seg = (((1u << L) - 1u) << (lane & ~static_cast<unsigned>(L - 1)));
+  const int total = B * N;
+  const int chunk = (total + gridDim.x - 1) / gridDim.x;
+  const int t0 = blockIdx.x * chunk, t1 = min(total, t0 + chunk);
+  for (int h0 = threadIdx.x / L; h0 < H; h0 += S) {
+    float a = 0.f;
+    int b = t0 < t1 ? t0 / N : 0;
+    for (int tok = t0; tok < t1; ++tok) {
+      const int bt = tok / N;
+      if (bt != b) {
+        float ar = a;
+#pragma unroll
+        for (int o = L / 2; o > 0; o >>= 1) ar = fmaxf(ar, __shfl_xor_sync(seg, ar, o));
+        if (li == 0) atomicMax(amax_bits + b * H + h0, __float_as_uint(ar));
+        a = 0.f;
+        b = bt;
+      }
+      const __nv_bfloat16* src = v + (static_cast<long long>(tok) * H + h0) * D + li * 16;
+      const uint4 r0 = __ldcs(reinterpret_cast<const uint4*>(src));
+      const uint4 r1 = __ldcs(reinterpret_cast<const uint4*>(src + 8));
+      const uint32_t w[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        a = fmaxf(a, fmaxf(fabsf(__uint_as_float(w[i] << 16)), fabsf(__uint_as_float(w[i] & 0xFFFF0000u))));
+    }
+    if (t0 < t1) {
+#pragma unroll
+      for (int o = L / 2; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(seg, a, o));
+      if (li == 0) atomicMax(amax_bits + b * H + h0, __float_as_uint(a));
+    }
+  }
+}
+
+// Position j of every aligned group of 16 keys of a V^T row holds key kVtKey(j).
+__host__ __device__ constexpr int vt_key(int j) { return 2 * (j >> 2) + (j & 1) + 8 * ((j >> 1) & 1); }
+
+// V [B, N, H, D] bf16 -> V^T codes [B, H, D, N] e4m3 (keys permuted within
+// groups of 16 as vt_key) with the per-(b, h) scale s = amax / 448: codes are
+// v * (448 / amax) rounded to nearest e4m3.  One CTA (256 threads) per (b, h,
+// 128-key block): the block's tokens go through shared memory and come out as
+// 16-byte rows of keys.  N % 16 == 0.
+__global__ void __launch_bounds__(256) quant_vt_e4m3_kernel(const __nv_bfloat16* __restrict__ v,
+                                                            const unsigned* __restrict__ amax_bits,
+                                                            uint8_t* __restrict__ vt, float* __restrict__ v_scale,
+                                                            int B, int N, int H, int nb) {
+  constexpr int D = 128, P = D + 8;   // row pitch in bf16 (16-byte pad)
+  __shared__ __align__(16) __nv_bfloat16 tile[128 * P];
+  const int blk = blockIdx.x % nb;
+  const int bh = blockIdx.x / nb;
+  const int h = bh % H, b = bh / H;
+  const int k0 = blk * 128;
+  const int nk = min(128, N - k0);
+  // load: 16 threads per token row (256 bytes), 16 rows per pass
+  for (int e = threadIdx.x; e < 128 * 16; e += 256) {
+    const int key = e / 16, c = (e % 16) * 8;
+    uint4 w = make_uint4(0u, 0u, 0u, 0u);
+    if (key < nk) w = __ldcs(reinterpret_cast<const uint4*>(v + ((static_cast<long long>(b) * N + k0 + key) * H + h) * D + c));
+    *reinterpret_cast<uint4*>(tile + key * P + c) = w;
+  }
+  __syncthreads();
+  const float amax = __uint_as_float(__ldg(amax_bits + bh));
+  const float s = __fdiv_rn(amax, 448.0f);
+  const float rcp = __fdiv_rn(448.0f, amax > 0.f ? amax : 1.0f);
+  if (blk == 0 && threadIdx.x == 0) v_scale[bh] = s;
+  // store: thread (g, d) writes positions 16 g .. 16 g + 15 of channel d's row
+  for (int e = threadIdx.x; e < 8 * D; e += 256) {
+    const int d = e % D, g = e / D;
+    if (16 * g >= nk) continue;
+    uint32_t out[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      float f[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int key = 16 * g + vt_key(4 * q + u);
+        f[u] = s > 0.f ? __fmul_rn(__bfloat162float(tile[key * P + d]), rcp) : 0.f;
+      }
+      const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(f[0], f[1]), __NV_SATFINITE, __NV_E4M3);
+      const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(f[2], f[3]), __NV_SATFINITE, __NV_E4M3);
+      out[q] = lo | (hi << 16);
+    }
+    __stcs(reinterpret_cast<uint4*>(vt + (static_cast<long long>(bh) * D + d) * N + k0 + 16 * g),
+           make_uint4(out[0], out[1], out[2], out[3]));
+  }
+}
+
 }  // namespace quant
 }  // namespace sol

@@ -24,6 +24,7 @@
 #include "select.cuh"
 #include "attn_pp.cuh"
 #include "quant.cuh"
+#include "attn_fp8.cuh"
 
 #ifndef SOL_ATTN_PINGPONG
 #define SOL_ATTN_PINGPONG 0   // 1: two query tiles per CTA in ping-pong (attn_pp.cuh)
@@ -50,7 +51,7 @@ int num_blocks(int N, int block) { return (N + block - 1) / block; }
 
 struct DeviceInfo {
   int sm_count = 0;
-  bool attn_attr = false, attn_pp_attr = false;
+  bool attn_attr = false, attn_pp_attr = false, attn_fp8_attr = false;
   bool select_attr[32] = {};   // score_topk / score_topp_kernel instantiations with the shared-memory opt-in set
 };
 DeviceInfo g_dev[kMaxDevices];
@@ -131,6 +132,32 @@ sol_status tile_blocks(const sol_shape& s, sol_tile tile, sol::BlockMap* out) {
 
 int blocks_of(const sol_shape& s, const sol::BlockMap& bm) {
   return bm.tw == 0 ? num_blocks(s.N, bm.block) : s.N / bm.block;
+}
+
+// e4m3 code maps of the FP8 attention: K codes [B, N, H, D] as 4-D (c, h, n, b)
+// with one 128-channel box per block of 128 tokens; V^T codes [B, H, D, N] as
+// 3-D (n, d, b * H + h) with one 128-key x 128-channel box.  Both 128-byte swizzled.
+sol_status make_fp8_maps(CUtensorMap* tk, CUtensorMap* tvt, const void* k8, const void* vt8, const sol_shape& s) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return SOL_ERR_CUDA;
+  cuuint64_t kd[4] = {static_cast<cuuint64_t>(s.D), static_cast<cuuint64_t>(s.H), static_cast<cuuint64_t>(s.N),
+                      static_cast<cuuint64_t>(s.B)};
+  cuuint64_t ks[3] = {static_cast<cuuint64_t>(s.D), static_cast<cuuint64_t>(s.H) * s.D,
+                      static_cast<cuuint64_t>(s.N) * s.H * s.D};
+  cuuint32_t kb[4] = {128, 1, 128, 1};
+  cuuint32_t e4[4] = {1, 1, 1, 1};
+  CUresult r = enc(tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(k8), kd, ks, kb, e4,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return SOL_ERR_CUDA;
+  cuuint64_t vd[3] = {static_cast<cuuint64_t>(s.N), static_cast<cuuint64_t>(s.D),
+                      static_cast<cuuint64_t>(s.B) * s.H};
+  cuuint64_t vs[2] = {static_cast<cuuint64_t>(s.N), static_cast<cuuint64_t>(s.D) * s.N};
+  cuuint32_t vb[3] = {128, 128, 1};
+  cuuint32_t e3[3] = {1, 1, 1};
+  r = enc(tvt, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(vt8), vd, vs, vb, e3, CU_TENSOR_MAP_INTERLEAVE_NONE,
+          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? SOL_OK : SOL_ERR_CUDA;
 }
 
 sol_status launch_status() { return cudaGetLastError() == cudaSuccess ? SOL_OK : SOL_ERR_CUDA; }
@@ -539,6 +566,97 @@ sol_status sol_dequant_unpack(const void* codes, const float* scales, int B, int
       sol::quant::dequant_unpack_kernel<64, sol::quant::kE4M3><<<g, threads, 0, stream>>>(cb, scales, ob, B, Nc, Hc, G,
                                                                                       split, g_stride_rows);
   }
+  return launch_status();
+}
+
+size_t sol_quant_attn_fp8_workspace_bytes(sol_shape s) {
+  if (!shape_ok(s)) return 0;
+  return (static_cast<size_t>(s.B) * s.H * sizeof(unsigned) + 15) / 16 * 16;
+}
+
+sol_status sol_quant_attn_fp8(const void* q, const void* k, const void* v, sol_shape s, void* q8, float* q_scale,
+                              void* k8, float* k_scale, void* vt8, float* v_scale, void* workspace,
+                              size_t workspace_bytes, cudaStream_t stream) {
+  if (!q || !k || !v || !q8 || !q_scale || !k8 || !k_scale || !vt8 || !v_scale || !workspace)
+    return SOL_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(q8) || !aligned16(k8) || !aligned16(vt8) ||
+      !aligned16(workspace))
+    return SOL_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(q_scale) % 8 || reinterpret_cast<uintptr_t>(k_scale) % 8 ||
+      reinterpret_cast<uintptr_t>(v_scale) % 4)
+    return SOL_ERR_INVALID_ARG;
+  if (!shape_ok(s)) return SOL_ERR_INVALID_ARG;
+  if (workspace_bytes < sol_quant_attn_fp8_workspace_bytes(s)) return SOL_ERR_INVALID_ARG;
+  if (s.D != 128 || s.N % 16 != 0) return SOL_ERR_UNSUPPORTED;
+  if (static_cast<long long>(s.B) * s.N * s.H >= 0x7fffffffll) return SOL_ERR_UNSUPPORTED;
+  DeviceInfo* di = nullptr;
+  if (sol_status st = device_info(&di)) return st;
+  const auto* qb = static_cast<const __nv_bfloat16*>(q);
+  const auto* kb = static_cast<const __nv_bfloat16*>(k);
+  const auto* vb = static_cast<const __nv_bfloat16*>(v);
+  const int threads = std::min(s.H * (s.D / 16), 512);
+  const unsigned grid = static_cast<unsigned>(std::min<long long>(static_cast<long long>(s.B) * s.N,
+                                                                  quant_grid(di, threads)));
+  sol::quant::quant_rows_e4m3_kernel<128><<<grid, threads, 0, stream>>>(qb, static_cast<uint8_t*>(q8), q_scale, s.B,
+                                                                        s.N, s.H);
+  sol::quant::quant_rows_e4m3_kernel<128><<<grid, threads, 0, stream>>>(kb, static_cast<uint8_t*>(k8), k_scale, s.B,
+                                                                        s.N, s.H);
+  auto* amax = static_cast<unsigned*>(workspace);
+  if (cudaMemsetAsync(amax, 0, static_cast<size_t>(s.B) * s.H * sizeof(unsigned), stream) != cudaSuccess)
+    return SOL_ERR_CUDA;
+  const int athreads = std::min(s.H * (s.D / 16), 256);
+  const unsigned agrid = static_cast<unsigned>(std::min<long long>(static_cast<long long>(s.B) * s.N,
+                                                                   quant_grid(di, athreads)));
+  sol::quant::head_amax_kernel<128><<<agrid, athreads, 0, stream>>>(vb, amax, s.B, s.N, s.H);
+  const int nb = num_blocks(s.N, 128);
+  const long long vgrid = static_cast<long long>(s.B) * s.H * nb;
+  if (vgrid > 0x7fffffffll) return SOL_ERR_UNSUPPORTED;
+  sol::quant::quant_vt_e4m3_kernel<<<static_cast<unsigned>(vgrid), 256, 0, stream>>>(
+      vb, amax, static_cast<uint8_t*>(vt8), v_scale, s.B, s.N, s.H, nb);
+  return launch_status();
+}
+
+sol_status sol_sparse_attn_fwd_fp8(const void* q8, const float* q_scale, const void* k8, const float* k_scale,
+                                   const void* vt8, const float* v_scale, const int32_t* idx, const int32_t* counts,
+                                   sol_shape s, int block, int topk, float softmax_scale, void* o, float* lse,
+                                   cudaStream_t stream) {
+  if (!q8 || !q_scale || !k8 || !k_scale || !vt8 || !v_scale || !idx || !o || !lse) return SOL_ERR_INVALID_ARG;
+  if (!aligned16(q8) || !aligned16(k8) || !aligned16(vt8) || !aligned16(idx) || !aligned16(o) || !aligned16(lse))
+    return SOL_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(q_scale) % 8 || reinterpret_cast<uintptr_t>(k_scale) % 8) return SOL_ERR_INVALID_ARG;
+  if (!shape_ok(s) || block <= 0) return SOL_ERR_INVALID_ARG;
+  const int nb = num_blocks(s.N, block);
+  if (topk < 1 || topk > nb) return SOL_ERR_INVALID_ARG;
+  if (!std::isfinite(softmax_scale)) return SOL_ERR_INVALID_ARG;
+  if (s.D != sol::attnfp8::kHeadDim || block != sol::attnfp8::kBlock || s.N % 16 != 0) return SOL_ERR_UNSUPPORTED;
+  const long long tiles = static_cast<long long>(s.B) * s.H * nb;
+  if (tiles > 0x7fffffffll) return SOL_ERR_UNSUPPORTED;
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(s.D));
+  DeviceInfo* di = nullptr;
+  if (sol_status st = device_info(&di)) return st;
+  CUtensorMap tk, tvt;
+  if (sol_status st = make_fp8_maps(&tk, &tvt, k8, vt8, s)) return st;
+  const size_t smem = sizeof(sol::attnfp8::Smem) + 1024;
+  if (!di->attn_fp8_attr) {
+    if (cudaFuncSetAttribute(sol::attnfp8::sparse_attn_fp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return SOL_ERR_CUDA;
+    di->attn_fp8_attr = true;
+  }
+  sol::attnfp8::Params p;
+  p.q = static_cast<const uint8_t*>(q8);
+  p.q_scale = q_scale;
+  p.k_scale = k_scale;
+  p.v_scale = v_scale;
+  p.idx = idx;
+  p.counts = counts;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.B = s.B; p.N = s.N; p.H = s.H; p.nb = nb; p.topk = topk;
+  p.num_tiles = static_cast<int>(tiles);
+  p.scale_log2 = scale * 1.4426950408889634f;
+  const int grid = static_cast<int>(std::min<long long>(tiles, di->sm_count));
+  sol::attnfp8::sparse_attn_fp8_kernel<<<grid, sol::attnfp8::kThreads, smem, stream>>>(tk, tvt, p);
   return launch_status();
 }
 

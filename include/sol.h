@@ -293,6 +293,39 @@ sol_status sol_dequant_unpack(const void* codes, const float* scales, int B, int
                               cudaStream_t stream);
 
 /*
+ * FP8 (e4m3) attention -- the Sol-Attn forward on e4m3 operands (the pages'
+ * runtime uses FP8 on its hot paths: ai-feiten.nl, "Videomodel MiniMax-H3
+ * rendert sneller dan afspelen", "Waar de snelheidswinst vandaan komt"; the
+ * formats are this library's).
+ *
+ * sol_quant_attn_fp8: bf16 q, k, v [B,N,H,D] (D == 128, N % 16 == 0) ->
+ *   q8, k8      e4m3 codes [B,N,H,D]; q_scale, k_scale fp32 [B,H,N], one per
+ *               (token, head) row: s = max|x| / 448, codes x * (448 / max|x|)
+ *               rounded to nearest even (an all-zero row: s = 0, zero codes);
+ *   vt8         e4m3 codes of V transposed, [B,H,D,N], the keys of every
+ *               aligned group of 16 stored in the order
+ *               0 1 8 9 2 3 10 11 4 5 12 13 6 7 14 15;
+ *   v_scale     fp32 [B,H], one per (b, h): s = max|v| / 448 over all tokens
+ *               and channels, codes v * (448 / max|v|);
+ *   workspace   device scratch of sol_quant_attn_fp8_workspace_bytes(s).
+ *   q_scale, k_scale 8-byte aligned; the others 16-byte aligned.
+ * sol_sparse_attn_fwd_fp8: the attention of sol_sparse_attn_fwd(_counts) on
+ *   the dequantised q = q8 * q_scale, k = k8 * k_scale, v = vt8^T * v_scale,
+ *   with e4m3 tensor-core products (fp32 accumulation) and the softmax weights
+ *   rounded to e4m3 for the P V product (relative error 2^-4 per weight; the
+ *   normaliser uses the unrounded weights).  counts may be NULL (every row uses
+ *   topk blocks).  block == 128; o bf16 [B,N,H,D], lse fp32 [B,H,N].
+ */
+size_t sol_quant_attn_fp8_workspace_bytes(sol_shape s);
+sol_status sol_quant_attn_fp8(const void* q, const void* k, const void* v, sol_shape s, void* q8, float* q_scale,
+                              void* k8, float* k_scale, void* vt8, float* v_scale, void* workspace,
+                              size_t workspace_bytes, cudaStream_t stream);
+sol_status sol_sparse_attn_fwd_fp8(const void* q8, const float* q_scale, const void* k8, const float* k_scale,
+                                   const void* vt8, const float* v_scale, const int32_t* idx, const int32_t* counts,
+                                   sol_shape s, int block, int topk, float softmax_scale, void* o, float* lse,
+                                   cudaStream_t stream);
+
+/*
  * sol_block_select_noalloc -- sol_block_select for callers that cannot
  * allocate device memory.  No counterpart on the pages: this is a convenience
  * of this library.

@@ -263,3 +263,25 @@ def test_quant_exchange_argument_checks(lib):
     assert unpack(FAKE, FAKE, 1, 48, 2, 128, 0, 0, 0, FAKE, 0, None) == INVALID     # G = 0
     assert unpack(FAKE, FAKE, 1, 48, 2, 128, 2, 0, 0, FAKE, 95, None) == INVALID    # stride < 96 rows
     assert unpack(FAKE, FAKE, 1, 48, 2, 32, 2, 0, 0, FAKE, 0, None) == UNSUPPORTED
+
+
+def test_fp8_argument_checks(lib):
+    ws = lib.sol_quant_attn_fp8_workspace_bytes
+    ws.restype = ctypes.c_size_t
+    ws.argtypes = [Shape]
+    assert ws(OK_SHAPE) == 16                                   # B * H = 2 fp32 words, rounded to 16 bytes
+    q = lib.sol_quant_attn_fp8
+    q.restype = ctypes.c_int
+    q.argtypes = [ctypes.c_void_p] * 3 + [Shape] + [ctypes.c_void_p] * 7 + [ctypes.c_size_t, ctypes.c_void_p]
+    s128 = Shape(1, 1024, 2, 128, 4, 16, 16)
+    assert q(FAKE, FAKE, FAKE, s128, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, None) == INVALID     # workspace
+    assert q(FAKE, FAKE, FAKE, s128, FAKE, None, FAKE, FAKE, FAKE, FAKE, FAKE, 16, None) == INVALID
+    assert q(FAKE, FAKE, FAKE, s128, FAKE, ctypes.c_void_p(0x10004), FAKE, FAKE, FAKE, FAKE, FAKE, 16, None) == INVALID
+    assert q(FAKE, FAKE, FAKE, OK_SHAPE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 16, None) == UNSUPPORTED  # D = 64
+    a = lib.sol_sparse_attn_fwd_fp8
+    a.restype = ctypes.c_int
+    a.argtypes = [ctypes.c_void_p] * 8 + [Shape, ctypes.c_int, ctypes.c_int, ctypes.c_float] + [ctypes.c_void_p] * 3
+    assert a(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, s128, 128, 0, 0.0, FAKE, FAKE, None) == INVALID  # k = 0
+    assert a(FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, None, s128, 128, 4, 0.0, FAKE, FAKE, None) == INVALID
+    assert a(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, s128, 64, 4, 0.0, FAKE, FAKE, None) == UNSUPPORTED
+    assert a(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, s128, 128, 4, float("inf"), FAKE, FAKE, None) == INVALID
