@@ -370,7 +370,7 @@ def sol_dequant_unpack(codes, scales, B, Nc, Hc, D, G, split, code, out, g_strid
 
 def sol_quant_attn_fp8(q, k, v, grid, out=None, stream=None):
     """e4m3 codes and scales of bf16 q, k, v [B, N, H, D] for sol_sparse_attn_fwd_fp8 (layouts in include/sol.h).
-    Returns a dict: q8, q_scale [B, H, N], k8, k_scale, vt8 [B, H, D, N], v_scale [B, H]."""
+    Returns a dict: q8, q_scale [B, H, N], k8, k_scale [B, H, nb], vt8 [B, H, D, N], v_scale [B, H]."""
     _cuda(q, "q"), _cuda(k, "k"), _cuda(v, "v")
     if q.dtype != torch.bfloat16 or k.dtype != torch.bfloat16 or v.dtype != torch.bfloat16:
         raise TypeError("q, k, v must be bf16")
@@ -381,7 +381,7 @@ def sol_quant_attn_fp8(q, k, v, grid, out=None, stream=None):
                "k8": torch.empty(k.shape, dtype=torch.uint8, device=dev),
                "vt8": torch.empty((s.B, s.H, s.D, s.N), dtype=torch.uint8, device=dev),
                "q_scale": torch.empty((s.B, s.H, s.N), dtype=torch.float32, device=dev),
-               "k_scale": torch.empty((s.B, s.H, s.N), dtype=torch.float32, device=dev),
+               "k_scale": torch.empty((s.B, s.H, -(-s.N // 128)), dtype=torch.float32, device=dev),
                "v_scale": torch.empty((s.B, s.H), dtype=torch.float32, device=dev)}
         ws = max(int(lib.sol_quant_attn_fp8_workspace_bytes(s)), 16)
         out["workspace"] = torch.empty(ws, dtype=torch.uint8, device=dev)

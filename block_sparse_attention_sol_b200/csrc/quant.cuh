@@ -361,5 +361,62 @@ __global__ void __launch_bounds__(256) quant_vt_e4m3_kernel(const __nv_bfloat16*
   }
 }
 
+// K [B, N, H, D] bf16 -> e4m3 codes [B, N, H, D] with one scale per (b, h, block
+// of 128 tokens), scales [B, H, nb]: s = max |k| over the block / 448, codes
+// k * (448 / max |k|).  One CTA (256 threads) per (b, h, block): the block's
+// rows go through shared memory, the CTA reduces their maximum, then writes the
+// codes row by row (16 channels per thread).
+__global__ void __launch_bounds__(256) quant_kblock_e4m3_kernel(const __nv_bfloat16* __restrict__ k,
+                                                                uint8_t* __restrict__ codes,
+                                                                float* __restrict__ scales, int B, int N, int H,
+                                                                int nb) {
+  constexpr int D = 128, P = D + 8;
+  __shared__ __align__(16) __nv_bfloat16 tile[128 * P];
+  __shared__ float red[8];
+  const int blk = blockIdx.x % nb;
+  const int bh = blockIdx.x / nb;
+  const int h = bh % H, b = bh / H;
+  const int k0 = blk * 128;
+  const int nk = min(128, N - k0);
+  float a = 0.f;
+  for (int e = threadIdx.x; e < 128 * 16; e += 256) {
+    const int key = e / 16, c = (e % 16) * 8;
+    uint4 w = make_uint4(0u, 0u, 0u, 0u);
+    if (key < nk) w = __ldcs(reinterpret_cast<const uint4*>(k + ((static_cast<long long>(b) * N + k0 + key) * H + h) * D + c));
+    *reinterpret_cast<uint4*>(tile + key * P + c) = w;
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      a = fmaxf(a, fmaxf(fabsf(__uint_as_float(u[i] << 16)), fabsf(__uint_as_float(u[i] & 0xFFFF0000u))));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = a;
+  __syncthreads();
+  a = red[0];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) a = fmaxf(a, red[w]);
+  const float s = __fdiv_rn(a, 448.0f);
+  const float rcp = __fdiv_rn(448.0f, a > 0.f ? a : 1.0f);
+  if (threadIdx.x == 0) scales[static_cast<long long>(bh) * nb + blk] = s;
+  for (int e = threadIdx.x; e < 128 * 8; e += 256) {
+    const int key = e / 8, seg = (e % 8) * 16;
+    if (key >= nk) continue;
+    uint32_t out[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      float f[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        f[u] = s > 0.f ? __fmul_rn(__bfloat162float(tile[key * P + seg + 4 * q + u]), rcp) : 0.f;
+      const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(f[0], f[1]), __NV_SATFINITE, __NV_E4M3);
+      const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(f[2], f[3]), __NV_SATFINITE, __NV_E4M3);
+      out[q] = lo | (hi << 16);
+    }
+    __stcs(reinterpret_cast<uint4*>(codes + ((static_cast<long long>(b) * N + k0 + key) * H + h) * D + seg),
+           make_uint4(out[0], out[1], out[2], out[3]));
+  }
+}
+
 }  // namespace quant
 }  // namespace sol

@@ -599,8 +599,10 @@ sol_status sol_quant_attn_fp8(const void* q, const void* k, const void* v, sol_s
                                                                   quant_grid(di, threads)));
   sol::quant::quant_rows_e4m3_kernel<128><<<grid, threads, 0, stream>>>(qb, static_cast<uint8_t*>(q8), q_scale, s.B,
                                                                         s.N, s.H);
-  sol::quant::quant_rows_e4m3_kernel<128><<<grid, threads, 0, stream>>>(kb, static_cast<uint8_t*>(k8), k_scale, s.B,
-                                                                        s.N, s.H);
+  const int nbk = num_blocks(s.N, 128);
+  if (static_cast<long long>(s.B) * s.H * nbk > 0x7fffffffll) return SOL_ERR_UNSUPPORTED;
+  sol::quant::quant_kblock_e4m3_kernel<<<static_cast<unsigned>(s.B * s.H * nbk), 256, 0, stream>>>(
+      kb, static_cast<uint8_t*>(k8), k_scale, s.B, s.N, s.H, nbk);
   auto* amax = static_cast<unsigned*>(workspace);
   if (cudaMemsetAsync(amax, 0, static_cast<size_t>(s.B) * s.H * sizeof(unsigned), stream) != cudaSuccess)
     return SOL_ERR_CUDA;

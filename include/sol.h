@@ -299,9 +299,11 @@ sol_status sol_dequant_unpack(const void* codes, const float* scales, int B, int
  * formats are this library's).
  *
  * sol_quant_attn_fp8: bf16 q, k, v [B,N,H,D] (D == 128, N % 16 == 0) ->
- *   q8, k8      e4m3 codes [B,N,H,D]; q_scale, k_scale fp32 [B,H,N], one per
- *               (token, head) row: s = max|x| / 448, codes x * (448 / max|x|)
- *               rounded to nearest even (an all-zero row: s = 0, zero codes);
+ *   q8, k8      e4m3 codes [B,N,H,D]; q_scale fp32 [B,H,N], one per (token,
+ *               head) row; k_scale fp32 [B,H,nb], one per (b, h, block of 128
+ *               tokens): s = max|x| over the row or block / 448, codes
+ *               x * (448 / max|x|) rounded to nearest even (all zero: s = 0,
+ *               zero codes);
  *   vt8         e4m3 codes of V transposed, [B,H,D,N], the keys of every
  *               aligned group of 16 stored in the order
  *               0 1 8 9 2 3 10 11 4 5 12 13 6 7 14 15;

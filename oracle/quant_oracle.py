@@ -90,14 +90,17 @@ def quant_roundtrip(x, kind: str) -> np.ndarray:
 
 # ----------------------------------------------------------------------------- FP8 attention inputs
 # Readings for the FP8 (e4m3) variant of the attention (the pages say only that
-# the runtime uses FP8; the formats are this library's): Q and K rows are
-# quantised like the exchange rows above (one scale per (token, head) row);
-# V gets one scale per (batch, head), s_v = max |v| over all its tokens and
-# channels / 448, codes v * (448 / max |v|) rounded to nearest e4m3.  The
+# the runtime uses FP8; the formats are this library's): Q rows are quantised
+# like the exchange rows above (one scale per (token, head) row); K gets one
+# scale per (batch, head, block of 128 tokens) and V one per (batch, head):
+# s = max |x| over the group / 448, codes x * (448 / max |x|) rounded to
+# nearest e4m3.  (e4m3 keeps values down to 2^-14 of a group's maximum normal,
+# so block- and head-wide scales cost no precision on these inputs, and a block
+# scale folds into the softmax's per-row factor.)  The
 # attention is then the exact softmax attention of the dequantised values
 # (code * scale, in fp64 here); the kernel's further rounding of P to e4m3 is
 # an approximation that the tests bound.
-__all__ += ["quantize_heads_e4m3", "fp8_attention_inputs", "VT_KEY_ORDER"]
+__all__ += ["quantize_heads_e4m3", "quantize_blocks_e4m3", "fp8_attention_inputs", "VT_KEY_ORDER"]
 
 # V is stored transposed, [B, H, D, N], with the keys of every aligned group of
 # 16 in this order (position j of the group holds key VT_KEY_ORDER[j]).
@@ -117,20 +120,38 @@ def quantize_heads_e4m3(v):
     return codes, s
 
 
+def quantize_blocks_e4m3(x, block: int = 128):
+    """x [B, N, H, D] -> (codes float64 [B, N, H, D], scales float32 [B, H, nb]), one scale per
+    (b, h, block of `block` consecutive tokens; the last block may be short)."""
+    x32 = np.asarray(x, dtype=np.float32)
+    B, N, H, D = x32.shape
+    nb = -(-N // block)
+    codes = np.zeros(x32.shape)
+    scales = np.zeros((B, H, nb), dtype=np.float32)
+    for i in range(nb):
+        seg = x32[:, i * block:(i + 1) * block]                      # [B, n_i, H, D]
+        c, sc = quantize_heads_e4m3(seg)
+        codes[:, i * block:(i + 1) * block] = c
+        scales[:, :, i] = sc
+    return codes, scales
+
+
 def fp8_attention_inputs(q, k, v):
     """Codes, scales and the dequantised (exact, fp64) Q, K, V of the FP8 attention.
 
-    Returns dict with q_codes, q_scales [B, H, N], k_codes, k_scales [B, H, N],
-    v_codes [B, N, H, D], v_scales [B, H], and q_deq, k_deq, v_deq (float64
-    [B, N, H, D], code * scale without further rounding)."""
+    Returns dict with q_codes, q_scales [B, H, N], k_codes, k_scales [B, H, nb]
+    (blocks of 128 tokens), v_codes [B, N, H, D], v_scales [B, H], and q_deq,
+    k_deq, v_deq (float64 [B, N, H, D], code * scale without further rounding)."""
     qc, qs = quantize_rows(q, "e4m3")                               # scales [B, N, H]
-    kc, ks = quantize_rows(k, "e4m3")
+    kc, ks = quantize_blocks_e4m3(k, 128)
     vc, vs = quantize_heads_e4m3(v)
+    N = kc.shape[1]
+    ks_tok = np.repeat(ks, 128, axis=2)[:, :, :N]                   # [B, H, N]
     return {
         "q_codes": qc, "q_scales": np.ascontiguousarray(np.swapaxes(qs, 1, 2)),
-        "k_codes": kc, "k_scales": np.ascontiguousarray(np.swapaxes(ks, 1, 2)),
+        "k_codes": kc, "k_scales": ks,
         "v_codes": vc, "v_scales": vs,
         "q_deq": qc * qs.astype(np.float64)[..., None],
-        "k_deq": kc * ks.astype(np.float64)[..., None],
+        "k_deq": kc * np.swapaxes(ks_tok, 1, 2).astype(np.float64)[..., None],
         "v_deq": vc * vs.astype(np.float64)[:, None, :, None],
     }

@@ -91,7 +91,11 @@ def test_head_scales_fp8_inputs():
             assert np.array_equal(codes[b, :, h], want)
             assert np.abs(codes[b, :, h]).max() == 448.0
     d = orc.fp8_attention_inputs(v, v, v)
-    assert d["q_scales"].shape == (2, 3, 48) and d["v_scales"].shape == (2, 3)
+    assert d["q_scales"].shape == (2, 3, 48) and d["v_scales"].shape == (2, 3) and d["k_scales"].shape == (2, 3, 1)
+    # K blocks of 128 tokens: with 48 tokens one block, so K's scales are V's and its codes too
+    assert np.array_equal(d["k_scales"][:, :, 0], s) and np.array_equal(d["k_codes"], codes)
+    kc, ks = orc.quantize_blocks_e4m3(np.concatenate([v, 2 * v, v], axis=1), 48)   # 3 blocks of 48
+    assert np.array_equal(ks[:, :, 1], 2 * s) and np.array_equal(kc[:, 48:96], codes)
     assert np.allclose(d["v_deq"], v, rtol=2.0 ** -4, atol=2.0 ** -10 * np.abs(v).max() / 448 * 2)
 
 
