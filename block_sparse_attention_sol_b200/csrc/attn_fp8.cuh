@@ -47,6 +47,10 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColO = 256, kColP = 384, kColQ = 416;
 constexpr float kRescaleLog2 = 2.5f;              // lazy-rescale threshold (log2 units)
 constexpr float kPOffsetLog2 = 6.0f;              // P = 2^(x - m + 6) <= 2^8.5 < 448
+// Of every 8 exponentials, this many run as a polynomial on the FMA pipe instead
+// of on MUFU (16 results per clock per SM, the bound once the FP8 MMAs take half
+// the bf16 time).
+constexpr int kPolyPer8 = 0;
 
 struct __align__(1024) Smem {
   uint8_t k[kSlots][kTileBytes];
@@ -357,7 +361,16 @@ sparse_attn_fp8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
           float x0, x1, x2, x3;
           f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[4 * i]), __uint_as_float(sr[4 * i + 1])), f0, nm0), x0, x1);
           f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[4 * i + 2]), __uint_as_float(sr[4 * i + 3])), f1, nm1), x2, x3);
-          const float p0 = ex2_approx(x0), p1 = ex2_approx(x1), p2 = ex2_approx(x2), p3 = ex2_approx(x3);
+          float p0, p1, p2, p3;
+          if ((i & 7) >= 8 - kPolyPer8) {
+            exp2_poly_pair(x0, x1, p0, p1);   // FMA pipe
+            exp2_poly_pair(x2, x3, p2, p3);
+          } else {
+            p0 = ex2_approx(x0);              // MUFU
+            p1 = ex2_approx(x1);
+            p2 = ex2_approx(x2);
+            p3 = ex2_approx(x3);
+          }
           acc0[i & 1] = f2_add(acc0[i & 1], f2_pack(p0, p1));
           acc1[i & 1] = f2_add(acc1[i & 1], f2_pack(p2, p3));
           // i = 2m: low half of column 4m + c4; i = 2m + 1: high half
