@@ -50,7 +50,7 @@ constexpr float kPOffsetLog2 = 6.0f;              // P = 2^(x - m + 6) <= 2^8.5 
 // Of every 8 exponentials, this many run as a polynomial on the FMA pipe instead
 // of on MUFU (16 results per clock per SM, the bound once the FP8 MMAs take half
 // the bf16 time).
-constexpr int kPolyPer8 = 0;
+constexpr int kPolyPer8 = 2;
 
 struct __align__(1024) Smem {
   uint8_t k[kSlots][kTileBytes];
