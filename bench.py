@@ -39,6 +39,7 @@ sys.path.insert(0, ROOT)
 from workloads import WORKLOADS, make_inputs  # noqa: E402
 
 L2_BYTES = 126 * 1024 * 1024
+FP32_LANES = 148 * 128                # fp32 FMA lanes of a B200 (148 SMs x 128)
 
 
 def load_peaks():
@@ -401,6 +402,8 @@ def run_ours(args, wl, world, rank, local):
         fp8["quantise_frac_hbm"] = fp8["quantise_GB/s"] / peaks["hbm_gbs"]
         fp8["kernel"] = "sol::attnfp8::sparse_attn_fp8_kernel"
 
+    clock_mhz = sampler.summary().get("sm_mhz") or 1965.0
+
     def stages(st, fused):
         """Per-stage rates.  Algorithmic bytes: prologue reads q_raw, k_raw and writes
         q, k (+ the block means when fused); the split selection reads q, k and writes
@@ -415,7 +418,11 @@ def run_ours(args, wl, world, rank, local):
                          "frac_hbm": pro_b / st["prologue"] / 1e6 / peaks["hbm_gbs"]},
             "select": {"ms": st["select"], "GB/s": sel_b / st["select"] / 1e6,
                        "frac_hbm": sel_b / st["select"] / 1e6 / peaks["hbm_gbs"],
-                       "scoring_TFLOP/s_fp32": score_flops / st["select"] / 1e9},
+                       "scoring_TFLOP/s_fp32": score_flops / st["select"] / 1e9,
+                       # the selection moves little and computes much: its roofline is the fp32
+                       # FMA rate, 148 SMs x 128 lanes x 2 FLOP at the sampled SM clock
+                       "bound": "alu", "fp32_peak_tflops": FP32_LANES * 2 * clock_mhz * 1e-6,
+                       "frac_fp32": score_flops / st["select"] / 1e9 / (FP32_LANES * 2 * clock_mhz * 1e-6)},
             "preparation": {"ms": prep_ms, "GB/s": (4 * io_bytes + idx_bytes) / prep_ms / 1e6,
                             "frac_hbm": (4 * io_bytes + idx_bytes) / prep_ms / 1e6 / peaks["hbm_gbs"]},
             "attention": {"ms": st["attention"], "TFLOP/s": flops / st["attention"] / 1e9,
