@@ -22,13 +22,9 @@
 #include "attn_sm100.cuh"
 #include "prologue.cuh"
 #include "select.cuh"
-#include "attn_pp.cuh"
 #include "quant.cuh"
 #include "attn_fp8.cuh"
 
-#ifndef SOL_ATTN_PINGPONG
-#define SOL_ATTN_PINGPONG 0   // 1: two query tiles per CTA in ping-pong (attn_pp.cuh)
-#endif
 
 namespace {
 
@@ -51,7 +47,7 @@ int num_blocks(int N, int block) { return (N + block - 1) / block; }
 
 struct DeviceInfo {
   int sm_count = 0;
-  bool attn_attr = false, attn_pp_attr = false, attn_fp8_attr = false;
+  bool attn_attr = false, attn_fp8_attr = false;
   bool select_attr[32] = {};   // score_topk / score_topp_kernel instantiations with the shared-memory opt-in set
 };
 DeviceInfo g_dev[kMaxDevices];
@@ -727,32 +723,6 @@ sol_status sparse_attn_impl(const void* q, const void* k, const void* v, const i
   if (s.D != sol::attn100::kHeadDim || bm.block != sol::attn100::kBlock) return SOL_ERR_UNSUPPORTED;
   const long long tiles = static_cast<long long>(s.B) * s.H * nb;
   if (tiles > 0x7fffffffll) return SOL_ERR_UNSUPPORTED;
-#if SOL_ATTN_PINGPONG
-  if (bm.tw == 0) {
-    CUtensorMap tq, tk, tv;
-    if (sol_status st = make_bshd_map(&tq, q, s)) return st;
-    if (sol_status st = make_bshd_map(&tk, k, s)) return st;
-    if (sol_status st = make_bshd_map(&tv, v, s)) return st;
-    const size_t smem = sizeof(sol::attnpp::Smem) + 1024;
-    if (!di->attn_pp_attr) {
-      if (cudaFuncSetAttribute(sol::attnpp::sparse_attn_pp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(smem)) != cudaSuccess)
-        return SOL_ERR_CUDA;
-      di->attn_pp_attr = true;
-    }
-    sol::attnpp::Params p;
-    p.idx = idx;
-    p.o = static_cast<__nv_bfloat16*>(o);
-    p.lse = lse;
-    p.B = s.B; p.N = s.N; p.H = s.H; p.nb = nb; p.topk = topk;
-    p.num_tiles = static_cast<int>(tiles);
-    p.num_pairs = static_cast<int>((tiles + 1) / 2);
-    p.scale_log2 = scale * 1.4426950408889634f;
-    const int grid = static_cast<int>(std::min<long long>(p.num_pairs, di->sm_count));
-    sol::attnpp::sparse_attn_pp_kernel<<<grid, sol::attnpp::kThreads, smem, stream>>>(tq, tk, tv, p);
-    return launch_status();
-  }
-#endif
   CUtensorMap tk, tv;
   if (bm.tw == 0) {
     if (sol_status st = make_bshd_map(&tk, k, s)) return st;
