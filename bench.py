@@ -332,6 +332,47 @@ def run_ours(args, wl, world, rank, local):
         qbytes = 4 * io_b + 3 * io_b // 2 + 2 * 4 * wl.B * wl.H * wl.N
         fp8 = {"quantise_ms": qms, "quantise_GB/s": qbytes / qms / 1e6,
                "attention_ms": ams, "attention_TFLOP/s": wl.selected_flops(topk) / ams / 1e9}
+    # Selection variants and tile blocks (opt-in, not part of `value`): each timed over
+    # a few launches after one untimed launch, on the same prologue outputs.
+    variants = None
+    if args.variants:
+        variants = {}
+        nrep = min(args.steps, 10)
+
+        def timed(fn):
+            fn()
+            a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize(dev)
+            a_.record(stream)
+            for _ in range(nrep):
+                out_ = fn()
+            b_.record(stream)
+            torch.cuda.synchronize(dev)
+            return a_.elapsed_time(b_) / nrep, out_
+
+        ms_plain, _ = timed(lambda: sol.sol_block_select_pooled(qbar, kbar, wl.grid, wl.block, topk, idx_out=idx))
+        ms_forced, _ = timed(lambda: sol.sol_block_select_pooled_ex(qbar, kbar, wl.grid, wl.block, topk, flags=3))
+        ms_topp, (idx_p, cnt_p) = timed(lambda: sol.sol_block_select_pooled_ex(qbar, kbar, wl.grid, wl.block, topk,
+                                                                               flags=4, top_p=0.9, softmax_scale=2.0))
+        ms_cnt, _ = timed(lambda: sol.sol_sparse_attn_fwd_counts(q, k, d["v"], idx_p, cnt_p, wl.grid, wl.block,
+                                                                 o=o, lse=lse))
+        kept = int(cnt_p.sum().item())
+        flops_cnt = 4 * wl.block * wl.block * wl.D * kept          # every block of this workload is full
+        variants["select_ms"] = {"plain": ms_plain, "forced_diagonal_first_frame": ms_forced,
+                                 "top_p_0.9_scale_2": ms_topp}
+        variants["attention_top_p_counts"] = {"ms": ms_cnt, "mean_count": kept / cnt_p.numel(),
+                                              "TFLOP/s": flops_cnt / ms_cnt / 1e9}
+        tile = (4, 4, 8) if wl.grid[0] % 4 == 0 and wl.grid[1] % 4 == 0 and wl.grid[2] % 8 == 0 else None
+        if tile is not None:
+            ms_tp, (qt, kt_, qbt, kbt) = timed(lambda: sol.sol_qk_prologue_pool_tiled(
+                d["q"], d["k"], d["gamma_q"], d["gamma_k"], wl.grid, tile, wl.rope_split, wl.rope_theta, wl.eps,
+                q_out=q, k_out=k))
+            idx_t = sol.sol_block_select_pooled(qbt, kbt, wl.grid, wl.block, topk)
+            ms_ta, _ = timed(lambda: sol.sol_sparse_attn_fwd_tiled(q, k, d["v"], idx_t, wl.grid, tile, o=o, lse=lse))
+            variants["tiles_4x4x8"] = {"prologue_pool_ms": ms_tp, "attention_ms": ms_ta,
+                                       "attention_TFLOP/s": wl.selected_flops(topk) / ms_ta / 1e9}
+        if sol.sol_check_device_status() != sol.SOL_OK:
+            raise RuntimeError("device-side error in the variant runs")
     # End to end through host buffers, the way a caller streams clips: the pipeline
     # copies each step's raw Q, K, V in from pinned host memory, runs the fused chain
     # and copies O and LSE back, with the next step's inputs crossing PCIe while the
@@ -457,6 +498,7 @@ def run_ours(args, wl, world, rank, local):
             "overlap": "double-buffered over clips: step i+1's inputs cross PCIe while step i computes",
             "serial_ms_per_step": e2e_serial_ms},
         "fp8_attention": fp8,
+        "variants": variants,
         "gpu_launches": (3 if args.chain == "fused" else 4) * args.steps,
         "clocks": clocks,
     }
@@ -568,6 +610,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="profiling runs: skip the end-to-end runs")
     ap.add_argument("--no-fp8", action="store_true", help="skip the FP8 attention comparison")
+    ap.add_argument("--variants", action="store_true",
+                    help="also time the selection variants, count-limited attention and 3-D tile blocks")
     ap.add_argument("--chain", choices=("fused", "split"), default="fused",
                     help="fused: prologue emits the block means (3 launches per step); split: the selection "
                          "pools q and k itself (4 launches)")
