@@ -43,6 +43,7 @@ __all__ = [
     "bf16_round", "rope_angles", "qk_prologue", "block_pool", "block_scores",
     "topk_blocks", "near_tie_rows", "block_select", "sparse_attention",
     "sparse_attention_rows", "selected_flops", "first_frame_blocks", "select_variant", "tiled_blocks",
+    "sparse_attention_backward",
 ]
 
 
@@ -300,6 +301,44 @@ def sparse_attention(q, k, v, idx, block, scale: float | None = None, units=None
         o[b, members[i], h, :] = oi
         lse[b, h, members[i]] = li
     return o, lse
+
+
+def sparse_attention_backward(q, k, v, idx, do, block, scale: float | None = None, counts=None):
+    """Gradients of step a5 with respect to q, k and v, given the output gradient do.
+
+    For the queries of block i of (b, h) and the keys m of its kept blocks,
+    with P = softmax(scale * q k^T) over those keys and O = P v:
+        dv_m += sum_n P_nm do_n
+        dP_nm = do_n . v_m
+        dS_nm = P_nm (dP_nm - sum_m' P_nm' dP_nm')      (softmax Jacobian; the
+                 inner sum equals do_n . O_n)
+        dq_n += scale * sum_m dS_nm k_m
+        dk_m += scale * sum_n dS_nm q_n
+    Keys kept by several query blocks accumulate contributions from all of them.
+    The method is used for inference only; this is the definition a backward
+    kernel would follow.  Returns (dq, dk, dv) float64 [B, N, H, D].
+    """
+    q, k, v, do = (np.asarray(x, np.float64) for x in (q, k, v, do))
+    B, N, H, D = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    members = _members(N, block)
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    for b in range(B):
+        for h in range(H):
+            for i, rows in enumerate(members):
+                kept = np.asarray(idx[b, h, i])[: None if counts is None else int(counts[b, h, i])]
+                cols = np.concatenate([members[j] for j in kept])
+                s_ = scale * (q[b, rows, h] @ k[b, cols, h].T)
+                p_ = np.exp(s_ - s_.max(axis=1, keepdims=True))
+                p_ /= p_.sum(axis=1, keepdims=True)
+                o_ = p_ @ v[b, cols, h]
+                dp = do[b, rows, h] @ v[b, cols, h].T
+                ds = p_ * (dp - np.sum(do[b, rows, h] * o_, axis=1, keepdims=True))
+                dq[b, rows, h] += scale * ds @ k[b, cols, h]
+                np.add.at(dk[:, :, h], (b, cols), scale * ds.T @ q[b, rows, h])
+                np.add.at(dv[:, :, h], (b, cols), p_.T @ do[b, rows, h])
+    return dq, dk, dv
 
 
 def selected_flops(idx, N: int, block: int, D: int) -> int:

@@ -13,6 +13,7 @@ import pytest
 import oracle
 import oracle.sol_oracle as so
 from tests import test_oracle_pins as pins
+from tests import test_oracle_backward as bpins
 from tests import test_oracle_quant as qpins
 from tests import test_oracle_tiles as tpins
 from tests import test_oracle_variants as vpins
@@ -115,6 +116,28 @@ def _quantize_levels_128(x, kind):
     return codes, (s * np.float32(127.0) / np.float32(128.0)).astype(np.float32)
 
 
+def _backward_softmax_jacobian_dropped(q, k, v, idx, do, block, scale=None, counts=None):
+    # dS = P * dP, without subtracting the row's P . dP: a plausible slip in the softmax gradient
+    q, k, v, do = (np.asarray(x, np.float64) for x in (q, k, v, do))
+    B, N, H, D = q.shape
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    members = so._members(N, block)
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    for b in range(B):
+        for h in range(H):
+            for i, rows in enumerate(members):
+                kept = np.asarray(idx[b, h, i])[: None if counts is None else int(counts[b, h, i])]
+                cols = np.concatenate([members[j] for j in kept])
+                s_ = scale * (q[b, rows, h] @ k[b, cols, h].T)
+                p_ = np.exp(s_ - s_.max(axis=1, keepdims=True))
+                p_ /= p_.sum(axis=1, keepdims=True)
+                ds = p_ * (do[b, rows, h] @ v[b, cols, h].T)
+                dq[b, rows, h] += scale * ds @ k[b, cols, h]
+                np.add.at(dk[:, :, h], (b, cols), scale * ds.T @ q[b, rows, h])
+                np.add.at(dv[:, :, h], (b, cols), p_.T @ do[b, rows, h])
+    return dq, dk, dv
+
+
 MUTATIONS = [
     ("qk_prologue", _prologue_rope_sign, [pins.test_prologue_hand_case]),
     ("rope_angles", _angles_axis_reversed, [pins.test_prologue_hand_case]),
@@ -130,6 +153,8 @@ MUTATIONS = [
     ("tiled_blocks", _tiles_rows_columns_swapped, [tpins.test_tiled_blocks_hand_case]),
     ("e4m3_round", _e4m3_no_subnormals, [qpins.test_e4m3_round_matches_torch]),
     ("quantize_rows", _quantize_levels_128, [qpins.test_scales_and_dequantize_hand_case]),
+    ("sparse_attention_backward", _backward_softmax_jacobian_dropped,
+     [lambda: bpins.test_backward_matches_autograd(False)]),
 ]
 
 
