@@ -373,6 +373,24 @@ def run_ours(args, wl, world, rank, local):
                                        "attention_TFLOP/s": wl.selected_flops(topk) / ms_ta / 1e9}
         if sol.sol_check_device_status() != sol.SOL_OK:
             raise RuntimeError("device-side error in the variant runs")
+    # Backward pass (opt-in, not part of `value`): CUDA-core kernels, fp32 arithmetic.
+    # FLOPs counted as 2.5 x the forward's selected FLOPs (five products against two).
+    backward = None
+    if args.backward:
+        dout = torch.randn(o.shape, device=dev, dtype=torch.float32).to(o.dtype)
+        sol.sol_sparse_attn_fwd(q, k, d["v"], idx, wl.grid, wl.block, o=o, lse=lse)
+        ws_b = torch.empty(max(int(sol.lib.sol_sparse_attn_bwd_workspace_bytes(shape, wl.block)), 16),
+                           dtype=torch.uint8, device=dev)
+        sol.sol_sparse_attn_bwd(q, k, d["v"], o, lse, dout, idx, wl.grid, wl.block, workspace=ws_b)
+        b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        b0.record(stream)
+        sol.sol_sparse_attn_bwd(q, k, d["v"], o, lse, dout, idx, wl.grid, wl.block, workspace=ws_b)
+        b1.record(stream)
+        torch.cuda.synchronize(dev)
+        bms = b0.elapsed_time(b1)
+        backward = {"ms": bms, "TFLOP/s": 2.5 * wl.selected_flops(topk) / bms / 1e9,
+                    "kernels": "sol::attnbwd (CUDA cores, fp32)"}
     # End to end through host buffers, the way a caller streams clips: the pipeline
     # copies each step's raw Q, K, V in from pinned host memory, runs the fused chain
     # and copies O and LSE back, with the next step's inputs crossing PCIe while the
@@ -499,6 +517,7 @@ def run_ours(args, wl, world, rank, local):
             "serial_ms_per_step": e2e_serial_ms},
         "fp8_attention": fp8,
         "variants": variants,
+        "backward": backward,
         "gpu_launches": (3 if args.chain == "fused" else 4) * args.steps,
         "clocks": clocks,
     }
@@ -610,6 +629,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="profiling runs: skip the end-to-end runs")
     ap.add_argument("--no-fp8", action="store_true", help="skip the FP8 attention comparison")
+    ap.add_argument("--backward", action="store_true", help="also time the backward pass (one call)")
     ap.add_argument("--variants", action="store_true",
                     help="also time the selection variants, count-limited attention and 3-D tile blocks")
     ap.add_argument("--chain", choices=("fused", "split"), default="fused",

@@ -19,6 +19,7 @@ Functions (same names as the C ABI):
     sol_dequant_unpack(codes, scales, B, Nc, Hc, D, G, split, code, out, ...)
     sol_quant_attn_fp8(q, k, v, grid) -> dict of e4m3 codes and scales
     sol_sparse_attn_fwd_fp8(fp8_inputs, idx, grid, block, counts=None, ...) -> (o, lse)
+    sol_sparse_attn_bwd(q, k, v, o, lse, dout, idx, grid, block, counts=None, ...) -> (dq, dk, dv) fp32
     sol_check_device_status(stream=None)
     sol_selftest_wait_timeout(limit_us, stream=None)
     sol_block_select_workspace_bytes(shape, block)
@@ -34,7 +35,7 @@ __all__ = [
     "SolError", "SolShape", "LIB_PATH", "lib",
     "sol_qk_prologue", "sol_block_select", "sol_block_select_workspace_bytes", "sol_sparse_attn_fwd",
     "sol_qk_prologue_pool", "sol_block_select_pooled", "sol_block_select_pooled_ex", "sol_sparse_attn_fwd_counts",
-    "SolSelectOpts", "SolTile", "sol_quant_pack", "sol_dequant_unpack", "sol_quant_attn_fp8", "sol_sparse_attn_fwd_fp8",
+    "SolSelectOpts", "SolTile", "sol_quant_pack", "sol_dequant_unpack", "sol_quant_attn_fp8", "sol_sparse_attn_fwd_fp8", "sol_sparse_attn_bwd",
     "SOL_CODE_INT8", "SOL_CODE_E4M3", "SOL_SPLIT_HEADS", "SOL_SPLIT_TOKENS", "sol_qk_prologue_pool_tiled", "sol_sparse_attn_fwd_tiled", "SOL_SELECT_FORCE_DIAGONAL", "SOL_SELECT_FORCE_FIRST_FRAME", "SOL_SELECT_TOP_P",
     "sol_check_device_status", "sol_selftest_wait_timeout", "sol_status_string", "sol_attention_chain",
     "SOL_OK", "SOL_ERR_INVALID_ARG", "SOL_ERR_UNSUPPORTED", "SOL_ERR_CUDA", "SOL_ERR_TIMEOUT",
@@ -105,6 +106,10 @@ lib.sol_quant_attn_fp8.restype = _I
 lib.sol_quant_attn_fp8.argtypes = [_P, _P, _P, SolShape, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
 lib.sol_sparse_attn_fwd_fp8.restype = _I
 lib.sol_sparse_attn_fwd_fp8.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, SolShape, _I, _I, _F, _P, _P, _P]
+lib.sol_sparse_attn_bwd_workspace_bytes.restype = _SZ
+lib.sol_sparse_attn_bwd_workspace_bytes.argtypes = [SolShape, _I]
+lib.sol_sparse_attn_bwd.restype = _I
+lib.sol_sparse_attn_bwd.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, SolShape, _I, _I, _F, _I, _P, _P, _P, _P, _SZ, _P]
 lib.sol_sparse_attn_fwd.restype = _I
 lib.sol_sparse_attn_fwd.argtypes = [_P, _P, _P, _P, SolShape, _I, _I, _F, _I, _P, _P, _P]
 lib.sol_check_device_status.restype = _I
@@ -412,6 +417,28 @@ def sol_sparse_attn_fwd_fp8(fp8, idx, grid, block, counts=None, softmax_scale=0.
                                      lse.data_ptr(), _stream_handle(stream))
     _check(st, "sol_sparse_attn_fwd_fp8")
     return o, lse
+
+
+def sol_sparse_attn_bwd(q, k, v, o, lse, dout, idx, grid, block, counts=None, softmax_scale=0.0, workspace=None,
+                        stream=None):
+    """Gradients of the block-sparse attention.  Returns (dq, dk, dv) fp32 [B, N, H, D]."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (lse, "lse"), (dout, "dout"), (idx, "idx")):
+        _cuda(t, n)
+    if idx.dtype != torch.int32 or (counts is not None and counts.dtype != torch.int32):
+        raise TypeError("idx and counts must be int32")
+    s = _shape(q, grid)
+    need = int(lib.sol_sparse_attn_bwd_workspace_bytes(s, int(block)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    dq, dk, dv = (torch.empty(q.shape, dtype=torch.float32, device=q.device) for _ in range(3))
+    st = lib.sol_sparse_attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                 dout.data_ptr(), idx.data_ptr(),
+                                 _cuda(counts, "counts").data_ptr() if counts is not None else None, s, int(block),
+                                 int(idx.shape[-1]), float(softmax_scale), _dtype_code(q), dq.data_ptr(), dk.data_ptr(),
+                                 dv.data_ptr(), _cuda(workspace, "workspace").data_ptr(), workspace.numel(),
+                                 _stream_handle(stream))
+    _check(st, "sol_sparse_attn_bwd")
+    return dq, dk, dv
 
 
 def sol_check_device_status(stream=None) -> int:

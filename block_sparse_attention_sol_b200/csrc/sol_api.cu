@@ -14,6 +14,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <type_traits>
 
 #include "../../include/sol.h"
 #include "sm100_ptx.cuh"
@@ -24,6 +25,7 @@
 #include "select.cuh"
 #include "quant.cuh"
 #include "attn_fp8.cuh"
+#include "attn_bwd.cuh"
 
 
 namespace {
@@ -655,6 +657,67 @@ sol_status sol_sparse_attn_fwd_fp8(const void* q8, const float* q_scale, const v
   p.scale_log2 = scale * 1.4426950408889634f;
   const int grid = static_cast<int>(std::min<long long>(tiles, di->sm_count));
   sol::attnfp8::sparse_attn_fp8_kernel<<<grid, sol::attnfp8::kThreads, smem, stream>>>(tk, tvt, p);
+  return launch_status();
+}
+
+size_t sol_sparse_attn_bwd_workspace_bytes(sol_shape s, int block) {
+  if (!shape_ok(s) || block <= 0) return 0;
+  const size_t bh = static_cast<size_t>(s.B) * s.H, nb = static_cast<size_t>(num_blocks(s.N, block));
+  auto r16 = [](size_t x) { return (x + 15) / 16 * 16; };
+  return r16(bh * s.N * sizeof(float)) + r16(bh * nb * nb * sizeof(int32_t)) + r16(bh * nb * sizeof(int32_t));
+}
+
+sol_status sol_sparse_attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                               const void* dout, const int32_t* idx, const int32_t* counts, sol_shape s, int block,
+                               int topk, float softmax_scale, sol_dtype dt, float* dq, float* dk, float* dv,
+                               void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  if (!q || !k || !v || !o || !lse || !dout || !idx || !dq || !dk || !dv || !workspace) return SOL_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(dq) ||
+      !aligned16(dk) || !aligned16(dv) || !aligned16(workspace))
+    return SOL_ERR_INVALID_ARG;
+  if (!shape_ok(s) || block <= 0) return SOL_ERR_INVALID_ARG;
+  if (dt != SOL_F32 && dt != SOL_BF16) return SOL_ERR_INVALID_ARG;
+  const int nb = num_blocks(s.N, block);
+  if (topk < 1 || topk > nb) return SOL_ERR_INVALID_ARG;
+  if (!std::isfinite(softmax_scale)) return SOL_ERR_INVALID_ARG;
+  if (workspace_bytes < sol_sparse_attn_bwd_workspace_bytes(s, block)) return SOL_ERR_INVALID_ARG;
+  if (s.D != 64 && s.D != 128) return SOL_ERR_UNSUPPORTED;
+  const long long rows = static_cast<long long>(s.B) * s.H * s.N;
+  const long long grid = (rows + sol::attnbwd::kWarps - 1) / sol::attnbwd::kWarps;
+  const long long tiles = static_cast<long long>(s.B) * s.H * nb;
+  if (grid > 0x7fffffffll || (tiles + 255) / 256 > 0x7fffffffll) return SOL_ERR_UNSUPPORTED;
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(s.D));
+  auto r16 = [](size_t x) { return (x + 15) / 16 * 16; };
+  const size_t bh = static_cast<size_t>(s.B) * s.H;
+  auto* base = static_cast<uint8_t*>(workspace);
+  auto* delta = reinterpret_cast<float*>(base);
+  auto* inv = reinterpret_cast<int32_t*>(base + r16(bh * s.N * sizeof(float)));
+  auto* inv_cnt = reinterpret_cast<int32_t*>(base + r16(bh * s.N * sizeof(float)) +
+                                             r16(bh * nb * static_cast<size_t>(nb) * sizeof(int32_t)));
+  const sol::attnbwd::Shape sh{s.B, s.N, s.H, block, nb, topk};
+  const dim3 g(static_cast<unsigned>(grid)), t(sol::attnbwd::kWarps * 32);
+  sol::attnbwd::bwd_invert_kernel<<<static_cast<unsigned>((tiles + 255) / 256), 256, 0, stream>>>(idx, counts, inv,
+                                                                                                    inv_cnt, sh);
+  auto run = [&](auto tag, auto dtag) {
+    using T = decltype(tag);
+    constexpr int D = decltype(dtag)::value;
+    const T* qq = static_cast<const T*>(q);
+    const T* kk = static_cast<const T*>(k);
+    const T* vv = static_cast<const T*>(v);
+    const T* oo = static_cast<const T*>(o);
+    const T* dd = static_cast<const T*>(dout);
+    sol::attnbwd::bwd_delta_kernel<T, D><<<g, t, 0, stream>>>(oo, dd, delta, sh);
+    sol::attnbwd::bwd_dq_kernel<T, D><<<g, t, 0, stream>>>(qq, kk, vv, dd, lse, delta, idx, counts, dq, sh, scale);
+    sol::attnbwd::bwd_dkdv_kernel<T, D><<<g, t, 0, stream>>>(qq, kk, vv, dd, lse, delta, inv, inv_cnt, dk, dv, sh,
+                                                             scale);
+  };
+  if (dt == SOL_BF16) {
+    if (s.D == 128) run(__nv_bfloat16{}, std::integral_constant<int, 128>{});
+    else run(__nv_bfloat16{}, std::integral_constant<int, 64>{});
+  } else {
+    if (s.D == 128) run(float{}, std::integral_constant<int, 128>{});
+    else run(float{}, std::integral_constant<int, 64>{});
+  }
   return launch_status();
 }
 

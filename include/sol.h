@@ -328,6 +328,25 @@ sol_status sol_sparse_attn_fwd_fp8(const void* q8, const float* q_scale, const v
                                    cudaStream_t stream);
 
 /*
+ * sol_sparse_attn_bwd -- gradients of sol_sparse_attn_fwd(_counts) (the method is
+ * used for inference; provided for completeness).  With P the softmax of
+ * scale * q k^T over the kept keys, recomputed from the forward's lse:
+ *   delta_n = do_n . o_n;  dS = P (do . v^T - delta);
+ *   dq = scale dS k;  dk = scale dS^T q;  dv = P^T do
+ * summed over every query block that kept a key block.
+ * q, k, v, o, dout : [B,N,H,D] (dtype dt); lse fp32 [B,H,N] from the forward;
+ * idx, counts (nullable) as for the forward; dq, dk, dv fp32 [B,N,H,D].
+ * workspace: sol_sparse_attn_bwd_workspace_bytes() (delta and the inverted
+ * selection index).  D in {64, 128}, any block; CUDA-core kernels, fp32 math;
+ * deterministic (no atomics).
+ */
+size_t sol_sparse_attn_bwd_workspace_bytes(sol_shape s, int block);
+sol_status sol_sparse_attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                               const void* dout, const int32_t* idx, const int32_t* counts, sol_shape s, int block,
+                               int topk, float softmax_scale, sol_dtype dt, float* dq, float* dk, float* dv,
+                               void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * sol_block_select_noalloc -- sol_block_select for callers that cannot
  * allocate device memory.  No counterpart on the pages: this is a convenience
  * of this library.

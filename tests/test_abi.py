@@ -285,3 +285,27 @@ def test_fp8_argument_checks(lib):
     assert a(FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, None, s128, 128, 4, 0.0, FAKE, FAKE, None) == INVALID
     assert a(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, s128, 64, 4, 0.0, FAKE, FAKE, None) == UNSUPPORTED
     assert a(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, s128, 128, 4, float("inf"), FAKE, FAKE, None) == INVALID
+
+
+def test_backward_argument_checks(lib):
+    ws = lib.sol_sparse_attn_bwd_workspace_bytes
+    ws.restype = ctypes.c_size_t
+    ws.argtypes = [Shape, ctypes.c_int]
+    need = ws(OK_SHAPE, 64)
+    assert need == 2 * 1024 * 4 + 2 * 16 * 16 * 4 + 2 * 16 * 4        # delta, inverted index, its counts
+    f = lib.sol_sparse_attn_bwd
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p] * 8 + [Shape, ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_int] + \
+        [ctypes.c_void_p] * 4 + [ctypes.c_size_t, ctypes.c_void_p]
+
+    def call(block=64, topk=4, ws_bytes=need, dq=FAKE, dt=0, shape=OK_SHAPE):
+        return f(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, shape, block, topk, 0.0, dt, dq, FAKE, FAKE, FAKE,
+                 ws_bytes, None)
+
+    assert call(ws_bytes=need - 4) == INVALID
+    assert call(topk=0) == INVALID
+    assert call(topk=17) == INVALID
+    assert call(dq=None) == INVALID
+    assert call(dq=MISALIGNED) == INVALID
+    assert call(dt=5) == INVALID
+    assert call(shape=Shape(1, 1024, 2, 96, 4, 16, 16), ws_bytes=1 << 20) == UNSUPPORTED
