@@ -15,7 +15,8 @@
  *  - Layouts: activations are [B, N, H, D] contiguous ("BSHD": token-major,
  *    then head, then channel).  Tokens are the latent video grid
  *    (grid_t, grid_h, grid_w) flattened in raster order, n = (t*grid_h + y)*grid_w + x.
- *    Blocks are runs of `block` consecutive tokens; the last may be short.
+ *    Blocks are runs of `block` consecutive tokens; the last may be short (the
+ *    *_tiled calls use 3-D tiles instead, see sol_tile).
  *  - Memory: every pointer is a DEVICE pointer on the current CUDA device,
  *    16-byte aligned, owned by the caller.  The library never allocates,
  *    frees or synchronises, except sol_check_device_status(), which
