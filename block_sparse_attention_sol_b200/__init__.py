@@ -38,6 +38,7 @@ __all__ = [
     "SolSelectOpts", "SolTile", "sol_quant_pack", "sol_dequant_unpack", "sol_quant_attn_fp8", "sol_sparse_attn_fwd_fp8", "sol_sparse_attn_bwd",
     "SOL_CODE_INT8", "SOL_CODE_E4M3", "SOL_SPLIT_HEADS", "SOL_SPLIT_TOKENS", "sol_qk_prologue_pool_tiled", "sol_sparse_attn_fwd_tiled", "SOL_SELECT_FORCE_DIAGONAL", "SOL_SELECT_FORCE_FIRST_FRAME", "SOL_SELECT_TOP_P",
     "sol_check_device_status", "sol_selftest_wait_timeout", "sol_status_string", "sol_attention_chain",
+    "sol_attention_chain_fused",
     "SOL_OK", "SOL_ERR_INVALID_ARG", "SOL_ERR_UNSUPPORTED", "SOL_ERR_CUDA", "SOL_ERR_TIMEOUT",
 ]
 
@@ -450,10 +451,22 @@ def sol_selftest_wait_timeout(limit_us: int, stream=None) -> None:
     _check(lib.sol_selftest_wait_timeout(int(limit_us), _stream_handle(stream)), "sol_selftest_wait_timeout")
 
 
+def sol_attention_chain_fused(q_raw, k_raw, v, gamma_q, gamma_k, grid, block, topk, rope_split=None,
+                              rope_theta=10000.0, eps=1e-6, softmax_scale=0.0, stream=None):
+    """The whole hot path on device tensors, three launches: the prologue that also
+    emits the block means -> scores and top-k from those means -> attention.
+    Returns (o, lse, idx, q, k), q and k being the prologue outputs."""
+    q, k, qbar, kbar = sol_qk_prologue_pool(q_raw, k_raw, gamma_q, gamma_k, grid, block, rope_split, rope_theta, eps,
+                                            stream=stream)
+    idx = sol_block_select_pooled(qbar, kbar, grid, block, topk, stream=stream)
+    o, lse = sol_sparse_attn_fwd(q, k, v, idx, grid, block, softmax_scale, stream=stream)
+    return o, lse, idx, q, k
+
+
 def sol_attention_chain(q_raw, k_raw, v, gamma_q, gamma_k, grid, block, topk, rope_split=None, rope_theta=10000.0,
                         eps=1e-6, softmax_scale=0.0, workspace=None, stream=None):
-    """The whole hot path on device tensors: prologue -> select -> attention.
-    Returns (o, lse, idx)."""
+    """The whole hot path on device tensors, four launches: prologue -> select
+    (pooling q and k itself) -> attention.  Returns (o, lse, idx)."""
     q, k = sol_qk_prologue(q_raw, k_raw, gamma_q, gamma_k, grid, rope_split, rope_theta, eps, stream=stream)
     idx = sol_block_select(q, k, grid, block, topk, workspace=workspace, stream=stream)
     o, lse = sol_sparse_attn_fwd(q, k, v, idx, grid, block, softmax_scale, stream=stream)

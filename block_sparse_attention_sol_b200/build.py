@@ -45,22 +45,8 @@ def _stale() -> bool:
 NO_SPILL_KERNELS = ("sparse_attn_fwd_kernel", "sparse_attn_fp8_kernel")
 
 
-# Kernels that split their registers between warpgroups with setmaxnreg: the split
-# is sized for this many registers per thread at launch, and setmaxnreg.inc would
-# wait for registers that do not exist if the launch got fewer.  The build refuses
-# any other count.
-LAUNCH_REGS = {}
-
-
 def _check_ptxas_report(report: str) -> None:
     lines = report.splitlines()
-    for name, regs in LAUNCH_REGS.items():
-        for i, line in enumerate(lines):
-            if "Compiling entry function" in line and name in line:
-                for follow in lines[i + 1:i + 4]:
-                    m = re.search(r"Used (\d+) registers", follow)
-                    if m and int(m.group(1)) != regs:
-                        raise RuntimeError(f"{name} launches with {m.group(1)} registers, its split needs {regs}")
     for name in NO_SPILL_KERNELS:
         found = False
         for i, line in enumerate(lines):

@@ -20,6 +20,7 @@
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
+#include "sm100_ptx.cuh"
 
 namespace sol {
 namespace attnbwd {
@@ -93,6 +94,10 @@ __global__ void __launch_bounds__(kWarps * 32) bwd_dq_kernel(const T* __restrict
   const int kt = row_count(counts, rowi, s.topk);
   for (int j = 0; j < kt; ++j) {
     const int blk = __ldg(list + j);
+    if (static_cast<unsigned>(blk) >= static_cast<unsigned>(s.nb)) {   // unusable id: skipped, reported
+      if (lane == 0) raise_bad_arg();
+      continue;
+    }
     const int m0 = blk * s.block, m1 = min(s.N, m0 + s.block);
     for (int m = m0; m < m1; ++m) {
       const size_t koff = (static_cast<size_t>(b) * s.N + m) * rs + h * D;
@@ -122,18 +127,26 @@ __global__ void __launch_bounds__(256) bwd_invert_kernel(const int32_t* __restri
   if (t >= static_cast<long long>(s.B) * s.H * s.nb) return;
   const int j = static_cast<int>(t % s.nb);
   const long long bh = t / s.nb;
+  // Every entry of every row is read, so that an id outside [0, nb) or an id a
+  // row repeats (which this index cannot represent) is reported, once, by the
+  // thread of key block 0 or of the repeated block.
   int c = 0;
+  bool bad = false;
   for (int i = 0; i < s.nb; ++i) {
     const size_t rowi = static_cast<size_t>(bh) * s.nb + i;
     const int32_t* list = idx + rowi * s.topk;
     const int kt = row_count(counts, rowi, s.topk);
-    for (int e = 0; e < kt; ++e)
-      if (__ldg(list + e) == j) {
-        inv[static_cast<size_t>(t) * s.nb + c++] = i;
-        break;
-      }
+    int hits = 0;
+    for (int e = 0; e < kt; ++e) {
+      const int id = __ldg(list + e);
+      hits += id == j ? 1 : 0;
+      bad |= j == 0 && static_cast<unsigned>(id) >= static_cast<unsigned>(s.nb);
+    }
+    if (hits > 0) inv[static_cast<size_t>(t) * s.nb + c++] = i;
+    bad |= hits > 1;
   }
   inv_cnt[t] = c;
+  if (bad) raise_bad_arg();
 }
 
 // dk, dv [B, N, H, D] fp32: one warp per key row.

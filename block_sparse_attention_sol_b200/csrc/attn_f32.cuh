@@ -9,6 +9,7 @@
 #pragma once
 #include <cstdint>
 #include "blocks.cuh"
+#include "sm100_ptx.cuh"
 
 namespace sol {
 namespace attnf32 {
@@ -38,6 +39,10 @@ __global__ void __launch_bounds__(kWarps * 32) sparse_attn_fwd_f32_kernel(
   float m = -INFINITY, l = 0.f;
   for (int j = 0; j < kt; ++j) {
     const int blk = list[j];
+    if (static_cast<unsigned>(blk) >= static_cast<unsigned>(nb)) {   // unusable id: skipped, reported
+      if (lane == 0) raise_bad_arg();
+      continue;
+    }
     const int len = bm.tw == 0 ? min(bm.block, N - blk * bm.block) : bm.block;
     for (int u = 0; u < len; ++u) {
       const int mk = block_token(bm, blk, u);

@@ -194,8 +194,14 @@ sparse_attn_fp8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
           if (use > 0 && !(ok = mbar_wait(&sm.slot_done[st], (use - 1) & 1, abort_flag, kSiteSlotFree))) break;
           const bool has_k = s < kt, has_v = s >= 2;
           mbar_arrive_expect_tx(&sm.kv_full[st], (has_k ? kTileBytes : 0) + (has_v ? kTileBytes : 0));
-          if (has_k) tma_load_4d(sm.k[st], &tm_k, &sm.kv_full[st], 0, h, __ldg(list + s) * kBlock, b);
-          if (has_v) tma_load_3d(sm.v[st], &tm_vt, &sm.kv_full[st], __ldg(list + s - 2) * kBlock, 0, b * p.H + h);
+          if (has_k) {
+            const int id = __ldg(list + s);
+            if (static_cast<unsigned>(id) >= static_cast<unsigned>(p.nb)) raise_bad_arg();
+            tma_load_4d(sm.k[st], &tm_k, &sm.kv_full[st], 0, h, usable_block(id, p.nb) * kBlock, b);
+          }
+          if (has_v)
+            tma_load_3d(sm.v[st], &tm_vt, &sm.kv_full[st], usable_block(__ldg(list + s - 2), p.nb) * kBlock, 0,
+                        b * p.H + h);
         }
       }
       for (uint32_t st = 0; st < kSlots; ++st)
@@ -318,7 +324,7 @@ sparse_attn_fp8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
       for (int j = 0; j < kt; ++j) {
         const uint32_t gg = g + j;
         const uint32_t buf = gg & 1;
-        const int blk = __ldg(list + j);
+        const int blk = usable_block(__ldg(list + j), p.nb);
         const float ksb = __ldg(ksc + blk);   // the block's K scale
         const uint32_t sl = sq + j;
         ok = mbar_wait(&sm.slot_done[sl % kSlots], (sl / kSlots) & 1, abort_flag, kSiteSDone);

@@ -165,8 +165,12 @@ sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
           if (use > 0 && !(ok = mbar_wait(&sm.slot_done[st], (use - 1) & 1, abort_flag, kSiteSlotFree))) break;
           const bool has_k = s < kt, has_v = s >= 2;
           mbar_arrive_expect_tx(&sm.kv_full[st], (has_k ? kTileBytes : 0) + (has_v ? kTileBytes : 0));
-          if (has_k) load_block(sm.k[st], &tm_k, &sm.kv_full[st], p, __ldg(list + s), h, b);
-          if (has_v) load_block(sm.v[st], &tm_v, &sm.kv_full[st], p, __ldg(list + s - 2), h, b);
+          if (has_k) {
+            const int id = __ldg(list + s);
+            if (static_cast<unsigned>(id) >= static_cast<unsigned>(p.nb)) raise_bad_arg();
+            load_block(sm.k[st], &tm_k, &sm.kv_full[st], p, usable_block(id, p.nb), h, b);
+          }
+          if (has_v) load_block(sm.v[st], &tm_v, &sm.kv_full[st], p, usable_block(__ldg(list + s - 2), p.nb), h, b);
         }
       }
       // Before the CTA exits, every load issued must have landed (slot s was
@@ -294,11 +298,11 @@ sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
       }
       float m0 = -INFINITY, m1 = -INFINITY;   // running max per row, log2 units (stale by < 2^8)
       float l0 = 0.f, l1 = 0.f;               // this thread's part of the running sums
-      int blk = __ldg(list);
+      int blk = usable_block(__ldg(list), p.nb);
       for (int j = 0; j < kt; ++j) {
         const uint32_t gg = g + j;
         const uint32_t buf = gg & 1;
-        const int blk_next = (j + 1 < kt) ? __ldg(list + j + 1) : 0;
+        const int blk_next = (j + 1 < kt) ? usable_block(__ldg(list + j + 1), p.nb) : 0;
         const uint32_t sl = sq + j;   // slot of K_j: its slot_done also means S_j is complete
         ok = mbar_wait(&sm.slot_done[sl % kSlots], (sl / kSlots) & 1, abort_flag, kSiteSDone);
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }

@@ -21,6 +21,7 @@
 #include <cuda_bf16.h>
 #include <cstdint>
 #include "blocks.cuh"
+#include "sm100_ptx.cuh"
 
 namespace sol {
 namespace prologue {
@@ -74,23 +75,32 @@ __device__ __forceinline__ void store_vec(__nv_bfloat16* p, const float (&y)[8])
 template <int V, int L>
 __device__ __forceinline__ void norm_rotate(float (&x)[V], const float (&g)[V], const float2 (&cs)[V / 2],
                                             unsigned seg, int D, float eps) {
-  float ss = 0.f;
-#pragma unroll
-  for (int e = 0; e < V; ++e) ss = fmaf(x[e], x[e], ss);
-#pragma unroll
-  for (int off = L / 2; off > 0; off >>= 1) ss += __shfl_xor_sync(seg, ss, off, L);
-  const float r = 1.0f / sqrtf(ss / static_cast<float>(D) + eps);
+  // packed fp32x2 sum of squares, rsqrt on MUFU (relative error ~2^-22, far inside
+  // the prologue's 2^-17 bound), packed gain products
+  uint64_t ss2 = 0ull;
 #pragma unroll
   for (int e = 0; e < V; e += 2) {
-    const float y0 = x[e] * r * g[e];
-    const float y1 = x[e + 1] * r * g[e + 1];
+    const uint64_t xe = f2_pack(x[e], x[e + 1]);
+    ss2 = f2_fma(xe, xe, ss2);
+  }
+  float sa, sb;
+  f2_unpack(ss2, sa, sb);
+  float ss = sa + sb;
+#pragma unroll
+  for (int off = L / 2; off > 0; off >>= 1) ss += __shfl_xor_sync(seg, ss, off, L);
+  const float r = rsqrtf(ss / static_cast<float>(D) + eps);
+  const uint64_t r2 = f2_pack(r, r);
+#pragma unroll
+  for (int e = 0; e < V; e += 2) {
+    float y0, y1;
+    f2_unpack(f2_mul(f2_mul(f2_pack(x[e], x[e + 1]), r2), f2_pack(g[e], g[e + 1])), y0, y1);
     x[e] = y0 * cs[e / 2].x - y1 * cs[e / 2].y;
     x[e + 1] = y0 * cs[e / 2].y + y1 * cs[e / 2].x;
   }
 }
 
 template <typename T, int D>
-__global__ void __launch_bounds__(256, sizeof(T) == 2 ? 3 : 4) qk_prologue_kernel(const Params p) {
+__global__ void __launch_bounds__(256, sizeof(T) == 2 ? 2 : 4) qk_prologue_kernel(const Params p) {
   extern __shared__ float2 tab[];   // [gt * dt/2 | gh * dh/2 | gw * dw/2] of (cos, sin)
   const int pt = p.dt / 2, ph = p.dh / 2, pw = p.dw / 2;
   for (int i = threadIdx.x; i < p.tab_total; i += blockDim.x) {

@@ -15,6 +15,7 @@
 #include <cstring>
 #include <mutex>
 #include <type_traits>
+#include <utility>
 
 #include "../../include/sol.h"
 #include "sm100_ptx.cuh"
@@ -47,8 +48,35 @@ bool shape_ok(const sol_shape& s) {
 
 int num_blocks(int N, int block) { return (N + block - 1) / block; }
 
+// Unique id of the calling thread's current CUDA context (0: none yet).  A
+// context created after cudaDeviceReset (or any other teardown of the primary
+// context) gets a new id, so per-device caches keyed by it never outlive the
+// context they were filled in.
+sol_status current_context_id(unsigned long long* id) {
+  static const auto fns = [] {
+    void* cur = nullptr;
+    void* get_id = nullptr;
+    cudaDriverEntryPointQueryResult q1, q2;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &cur, cudaEnableDefault, &q1) != cudaSuccess ||
+        q1 != cudaDriverEntryPointSuccess)
+      cur = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &get_id, cudaEnableDefault, &q2) != cudaSuccess ||
+        q2 != cudaDriverEntryPointSuccess)
+      get_id = nullptr;
+    return std::make_pair(reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(cur),
+                          reinterpret_cast<PFN_cuCtxGetId_v12000>(get_id));
+  }();
+  if (fns.first == nullptr || fns.second == nullptr) return SOL_ERR_CUDA;
+  CUcontext ctx = nullptr;
+  if (fns.first(&ctx) != CUDA_SUCCESS) return SOL_ERR_CUDA;
+  *id = 0;
+  if (ctx != nullptr && fns.second(ctx, id) != CUDA_SUCCESS) return SOL_ERR_CUDA;
+  return SOL_OK;
+}
+
 struct DeviceInfo {
   int sm_count = 0;
+  unsigned long long ctx_id = 0;   // context the attribute flags below were set in
   bool attn_attr = false, attn_fp8_attr = false;
   bool select_attr[32] = {};   // score_topk / score_topp_kernel instantiations with the shared-memory opt-in set
 };
@@ -58,8 +86,15 @@ std::mutex g_dev_mu;
 sol_status device_info(DeviceInfo** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SOL_ERR_CUDA;
+  unsigned long long ctx = 0;
+  if (sol_status st = current_context_id(&ctx)) return st;
   std::lock_guard<std::mutex> lock(g_dev_mu);
   DeviceInfo& d = g_dev[dev];
+  if (ctx == 0 || ctx != d.ctx_id) {   // kernel attributes belong to a context: set them again in this one
+    d.attn_attr = d.attn_fp8_attr = false;
+    for (bool& f : d.select_attr) f = false;
+    d.ctx_id = ctx;
+  }
   if (d.sm_count == 0) {
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
@@ -352,7 +387,7 @@ sol_status sol_qk_prologue(const void* q_raw, const void* k_raw, void* q_out, vo
   while (b) { const int r = a % b; a = b; b = r; }
   const long long unit = s.H / a;                       // CTAs per whole set of heads
   const long long needed = (static_cast<long long>(p.tokens) * s.H + groups_per_cta - 1) / groups_per_cta;
-  const long long target = static_cast<long long>(dt == SOL_BF16 ? 3 : 4) * di->sm_count;   // one resident wave
+  const long long target = static_cast<long long>(dt == SOL_BF16 ? 2 : 4) * di->sm_count;   // one resident wave (the kernel's launch bound)
   long long grid_ll = std::min(needed, target);
   grid_ll = (grid_ll + unit - 1) / unit * unit;
   if (grid_ll > 0x7fffffffll) return SOL_ERR_UNSUPPORTED;
@@ -828,19 +863,26 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[SOL_NOALLOC_SCR
 
 namespace {
 void* g_noalloc_ptr[kMaxDevices] = {};
+unsigned long long g_noalloc_ctx[kMaxDevices] = {};
 std::mutex g_noalloc_mu;
 
 // Host code may not pass g_noalloc_scratch itself to a kernel (on the host it
 // names a stand-in, not device memory): look up its device address once per
-// device, with that device current.
+// device and context, with that device current.  The address is cached with
+// the id of the context it was looked up in; a new context on the device (after
+// cudaDeviceReset, for instance) looks it up again.
 sol_status noalloc_scratch(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SOL_ERR_CUDA;
+  unsigned long long ctx = 0;
+  if (sol_status st = current_context_id(&ctx)) return st;
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (g_noalloc_ptr[dev] == nullptr) {
+  if (g_noalloc_ptr[dev] == nullptr || ctx == 0 || ctx != g_noalloc_ctx[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return SOL_ERR_CUDA;
+    if (sol_status st = current_context_id(&ctx)) return st;   // the lookup made the context current if it was not
     g_noalloc_ptr[dev] = p;
+    g_noalloc_ctx[dev] = ctx;
   }
   *out = g_noalloc_ptr[dev];
   return SOL_OK;

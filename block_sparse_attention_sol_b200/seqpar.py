@@ -16,7 +16,8 @@ the attention output as FP8, about half the inter-GPU bytes of bf16
 Every scale belongs to one (token, head) row, so the values that reach the
 attention do not depend on G.  The exchange itself goes through a Transport:
 CollectiveTransport (torch.distributed all_to_all_single: NCCL over NVLink on
-GPUs) or LocalTransport (G = 1).  Each exchange buffer is laid out
+GPUs), HostStagedTransport (the same collective on host copies, for gloo) or
+LocalTransport (G = 1).  Each exchange buffer is laid out
 [G][...] so that slice g is exactly what rank g receives (ExchangePlan).
 """
 from __future__ import annotations
@@ -28,7 +29,8 @@ import torch
 from . import (SOL_CODE_E4M3, SOL_CODE_INT8, SOL_SPLIT_HEADS, SOL_SPLIT_TOKENS, sol_block_select_pooled,
                sol_dequant_unpack, sol_qk_prologue_pool, sol_quant_pack, sol_sparse_attn_fwd)
 
-__all__ = ["ExchangePlan", "Transport", "CollectiveTransport", "LocalTransport", "SeqParallelAttention"]
+__all__ = ["ExchangePlan", "Transport", "CollectiveTransport", "HostStagedTransport", "LocalTransport",
+           "SeqParallelAttention"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -109,6 +111,22 @@ class CollectiveTransport(Transport):
 
     def all_to_all(self, recv, send):
         torch.distributed.all_to_all_single(recv, send, group=self.group)
+
+
+class HostStagedTransport(Transport):
+    """all_to_all through host memory: a device -> host copy of `send`,
+    torch.distributed all_to_all_single on the host tensors, a host -> device
+    copy into `recv`.  For process groups whose backend moves only host memory
+    (gloo), e.g. ranks that share one GPU; no peer memory is touched."""
+
+    def __init__(self, group=None):
+        self.group = group
+
+    def all_to_all(self, recv, send):
+        host_send = send.cpu()
+        host_recv = torch.empty_like(host_send)
+        torch.distributed.all_to_all_single(host_recv, host_send, group=self.group)
+        recv.copy_(host_recv)
 
 
 class LocalTransport(Transport):

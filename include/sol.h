@@ -207,7 +207,13 @@ sol_status sol_block_select_pooled_ex(const float* qbar, const float* kbar, sol_
  * idx[b,h,i,0..topk-1]:
  *   l_m = scale * q_n . k_m;  o_n = sum_m softmax(l)_m v_m;  lse_n = ln sum_m exp(l_m).
  * q, k, v : [B,N,H,D] (dtype dt).  idx : int32 [B,H,nb,topk], distinct ids in
- *           [0, nb) per row (any order; not checked).
+ *           [0, nb) per row (any order).  An id outside [0, nb) is never used
+ *           to address memory: the fp32 kernel skips it, the tensor-core
+ *           kernels read block 0 in its place, and either way the device error
+ *           word is set, which sol_check_device_status() reports as
+ *           SOL_ERR_INVALID_ARG (the outputs of that call are then undefined).
+ *           Repeated ids are not detected here: the block is attended once per
+ *           occurrence.
  * o       : [B,N,H,D] (dtype dt).  lse : fp32 [B,H,N], natural log, scale included.
  * softmax_scale <= 0 selects 1/sqrt(D).
  * bf16: D == 128 and block == 128 (tcgen05 tensor-core kernel, fp32 accumulate,
@@ -337,6 +343,10 @@ sol_status sol_sparse_attn_fwd_fp8(const void* q8, const float* q_scale, const v
  * summed over every query block that kept a key block.
  * q, k, v, o, dout : [B,N,H,D] (dtype dt); lse fp32 [B,H,N] from the forward;
  * idx, counts (nullable) as for the forward; dq, dk, dv fp32 [B,N,H,D].
+ * A row that repeats an id, or holds an id outside [0, nb), sets the device
+ * error word (sol_check_device_status() then returns SOL_ERR_INVALID_ARG) and
+ * the gradients of that call are undefined: the inverted index behind dk and
+ * dv records each (query block, key block) pair once.
  * workspace: sol_sparse_attn_bwd_workspace_bytes() (delta and the inverted
  * selection index).  D in {64, 128}, any block; CUDA-core kernels, fp32 math;
  * deterministic (no atomics).
@@ -364,8 +374,12 @@ sol_status sol_sparse_attn_bwd(const void* q, const void* k, const void* v, cons
  *    SOL_NOALLOC_SCRATCH_BYTES are rejected with SOL_ERR_UNSUPPORTED before
  *    anything is launched (the five video workloads need at most 33.4 MB).
  *  - First call per device: it looks up the array's device address
- *    (cudaGetSymbolAddress) with that device current and caches it; make
- *    that first call before any stream capture.  A failed lookup returns
+ *    (cudaGetSymbolAddress) with that device current and caches it together
+ *    with the id of the current CUDA context; make that first call before any
+ *    stream capture.  If the context changes (cudaDeviceReset, or another
+ *    teardown of the device's primary context, followed by new work), the next
+ *    call sees a new context id and looks the address up again: that call,
+ *    too, must come before any stream capture.  A failed lookup returns
  *    SOL_ERR_CUDA.
  *  - Sharing: every call on a device uses the same array and it keeps the
  *    last call's contents.  Nothing in it needs to start at zero (the pooling

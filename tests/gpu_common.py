@@ -18,7 +18,11 @@ Tolerances (written here once, used by every GPU test):
 from __future__ import annotations
 
 import functools
+import hashlib
+import json
 import math
+import os
+import time
 
 import numpy as np
 import torch
@@ -167,3 +171,50 @@ def check_attention(o_gpu, lse_gpu, q, k, v, idx, block, units, fp32: bool):
 
 def scale_of(D):
     return 1.0 / math.sqrt(D)
+
+
+# ---------------------------------------------------------------- parity record
+# The GPU parity tests write what they measured (rows compared, near-tie rows,
+# rows that differ, output errors) to tests/parity_record.json, one entry per
+# (workload, path), stamped with a hash of the kernel sources they ran, so the
+# counts the selection rule allows are reported and not only asserted.
+RECORD_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "parity_record.json")
+_ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def kernel_sources_sha256() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(_ROOT, "block_sparse_attention_sol_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    with open(os.path.join(_ROOT, "include", "sol.h"), "rb") as f:
+        h.update(f.read())
+    return h.hexdigest()
+
+
+def record_parity(key: str, **fields) -> None:
+    rec = {}
+    if os.path.exists(RECORD_PATH):
+        with open(RECORD_PATH) as f:
+            rec = json.load(f)
+    rec.setdefault("about", "written by the -m gpu parity tests (tests/test_gpu_workloads.py): per workload and "
+                            "path, the selection rows compared with the oracle, the near-tie rows among them (oracle "
+                            "k-th and (k+1)-th scores closer than 1e-4 relative, or than the chain's prologue band), "
+                            "the rows whose ids differ (allowed only among near-tie rows), and the attention errors")
+    entry = {k: (float(v) if isinstance(v, (np.floating, float)) else int(v) if isinstance(v, (np.integer,)) else v)
+             for k, v in fields.items()}
+    entry["kernel_sources_sha256"] = kernel_sources_sha256()
+    entry["when"] = time.strftime("%Y-%m-%dT%H:%M:%SZ", time.gmtime())
+    try:
+        entry["device"] = torch.cuda.get_device_name(0)
+    except Exception:
+        pass
+    rec.setdefault("entries", {})[key] = entry
+    rec["entries"] = dict(sorted(rec["entries"].items()))
+    tmp = RECORD_PATH + ".tmp"
+    with open(tmp, "w") as f:
+        json.dump(rec, f, indent=1)
+        f.write("\n")
+    os.replace(tmp, RECORD_PATH)

@@ -50,3 +50,35 @@ def test_backward_dv_closed_form_single_block():
     p = np.exp(s - s.max(axis=1, keepdims=True))
     p /= p.sum(axis=1, keepdims=True)
     assert np.allclose(dv[0, :, 0], p.T @ do[0, :, 0], rtol=0, atol=1e-13)
+
+
+def test_repeated_id_means_the_block_counts_twice():
+    """A row that lists a key block twice attends to its keys twice: the
+    oracle's forward equals dense attention over the concatenated key list
+    (torch SDPA in float64 over [K_0, K_1, K_1], closed form of the multiset),
+    and its backward equals autograd of that forward.  The library rejects such
+    rows in the backward (its inverted index records each pair once), so this
+    pins the definition a caller's repeated id would get, not the kernels."""
+    rng = np.random.default_rng(23)
+    B, N, H, D, block = 1, 16, 1, 4, 8            # 2 blocks
+    q, k, v, do = (rng.standard_normal((B, N, H, D)) for _ in range(4))
+    idx = np.array([[[[0, 1, 1], [1, 0, 0]]]], dtype=np.int32)
+    scale = 0.5
+    o, lse = orc.sparse_attention(q, k, v, idx, block, scale)
+    qt, kt, vt = (torch.tensor(x, dtype=torch.float64, requires_grad=True) for x in (q, k, v))
+    outs = []
+    for i in range(2):
+        rows = slice(i * block, (i + 1) * block)
+        cols = np.concatenate([np.arange(j * block, (j + 1) * block) for j in idx[0, 0, i]])
+        qi = qt[0, rows, 0][None, None]
+        kj, vj = kt[0, cols, 0][None, None], vt[0, cols, 0][None, None]
+        outs.append(torch.nn.functional.scaled_dot_product_attention(qi, kj, vj, scale=scale)[0, 0])
+        logits = scale * (q[0, rows, 0] @ k[0, cols, 0].T)
+        m = logits.max(axis=1)
+        assert np.allclose(lse[0, 0, rows], m + np.log(np.exp(logits - m[:, None]).sum(axis=1)), rtol=0, atol=1e-13)
+    ot = torch.cat(outs)
+    assert np.allclose(o[0, :, 0], ot.detach().numpy(), rtol=0, atol=1e-13)
+    ot.backward(torch.tensor(do[0, :, 0]))
+    got = orc.sparse_attention_backward(q, k, v, idx, do, block, scale)
+    for g, t in zip(got, (qt, kt, vt)):
+        assert np.allclose(g, t.grad.numpy(), rtol=0, atol=1e-12)
