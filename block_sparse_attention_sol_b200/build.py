@@ -43,10 +43,21 @@ def _stale() -> bool:
 
 # Kernels whose spilling would silently cost performance: the build refuses them.
 NO_SPILL_KERNELS = ("sparse_attn_fwd_kernel", "sparse_attn_fp8_kernel")
+# Register ceilings that launches need: a CTA's warps are spread over the SM's four
+# sub-partitions of 16 K registers each, so 10 warps (3 on some sub-partitions) get
+# at most 168 per thread; a kernel built above that fails to launch.
+MAX_REGS = {"sparse_attn_fwd_kernel": 168, "sparse_attn_fp8_kernel": 168}
 
 
 def _check_ptxas_report(report: str) -> None:
     lines = report.splitlines()
+    for name, cap in MAX_REGS.items():
+        for i, line in enumerate(lines):
+            if "Compiling entry function" in line and name in line:
+                for follow in lines[i + 1:i + 4]:
+                    m = re.search(r"Used (\d+) registers", follow)
+                    if m and int(m.group(1)) > cap:
+                        raise RuntimeError(f"{name} uses {m.group(1)} registers, more than the {cap} a launch allows")
     for name in NO_SPILL_KERNELS:
         found = False
         for i, line in enumerate(lines):

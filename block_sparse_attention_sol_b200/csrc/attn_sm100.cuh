@@ -25,7 +25,8 @@
 //               Online softmax in the exp2 domain with a lazy rescale (O is
 //               rescaled only when the running max grows by more than 2^8); P
 //               is written to TMEM as bf16 once PV of the previous step has
-//               completed (single P buffer); epilogue O / l -> bf16, LSE.
+//               completed (single P buffer); epilogue O / l -> bf16 with
+//               16-byte stores, and LSE.
 // TMEM columns: S0 [0,128) S1 [128,256) O [256,384) P [384,448) Q [448,512).
 // Shared memory: K 3 x 32 KB, V 3 x 32 KB.
 //
@@ -435,13 +436,38 @@ sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.o_free);
+      // The four threads of a row hold its channel pairs 8i + 2c (thread c); a 4 x 4
+      // exchange per group of four i gives thread c the 16 contiguous bytes of
+      // channels 8 (4a + c) .. + 7, which it stores in one instruction.
+      uint4 seg[2][4];
+#pragma unroll
+      for (int u = 0; u < 2; ++u)
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+          uint32_t got[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {   // round k: send pair 4a + (c4 - k) & 3, receive from thread (c4 + k) & 3
+            const int sidx = (c4 - k) & 3;
+            const uint32_t send = sidx == 0 ? ob[u][4 * a] : sidx == 1 ? ob[u][4 * a + 1]
+                                : sidx == 2 ? ob[u][4 * a + 2] : ob[u][4 * a + 3];
+            got[k] = __shfl_sync(0xffffffffu, send, (lane & ~3) | ((c4 + k) & 3));
+          }
+          // got[k] is the pair of channels 8 (4a + c4) + 2 ((c4 + k) & 3): put it in place
+          uint32_t w[4];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const int k = (c - c4) & 3;
+            w[c] = k == 0 ? got[0] : k == 1 ? got[1] : k == 2 ? got[2] : got[3];
+          }
+          seg[u][a] = make_uint4(w[0], w[1], w[2], w[3]);
+        }
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
         const int n = block_token(p.bm, qb, row0 + 8 * u);
         if (n < p.N) {
-          uint32_t* dst = reinterpret_cast<uint32_t*>(p.o + ((static_cast<size_t>(b) * p.N + n) * p.H + h) * kHeadDim);
+          uint4* dst = reinterpret_cast<uint4*>(p.o + ((static_cast<size_t>(b) * p.N + n) * p.H + h) * kHeadDim);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) dst[4 * i + c4] = ob[u][i];
+          for (int a = 0; a < 4; ++a) dst[4 * a + c4] = seg[u][a];
           if (c4 == 0)
             p.lse[(static_cast<size_t>(b) * p.H + h) * p.N + n] =
                 ((u ? m1 : m0) + __log2f(u ? l1 : l0)) * 0.69314718055994531f;

@@ -11,10 +11,11 @@
 //           each thread computes 4 rows x 4 keys of a 128-key chunk: 16-byte
 //           shared loads, rows broadcast across the warp, keys 32 apart.
 //   top-k:  per row, the k largest scores, exact ties to the lower j, written in
-//           ascending j.  A warp holds two rows' order-preserving keys in
-//           registers, finds each row's k-th largest by a most-significant-bit-
-//           first search of the 32-bit key space (the two searches interleaved),
-//           then compacts the winners in ascending j with ballots.
+//           ascending j.  A warp holds four rows' order-preserving keys in
+//           registers (two for nb > 1024), finds each row's threshold by a
+//           most-significant-bit-first search of the 32-bit key space (the
+//           searches interleaved; a row stops once exactly k keys pass), then
+//           compacts the winners in ascending j with ballots.
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -89,31 +90,44 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// The k-th largest key of a row held as KPL keys per lane (key j at lane j % 32,
-// slot j / 32; 0 pads, below every real key), then the row's ids with key above
-// it, plus the first (topk - count above) with key equal to it, in ascending j.
-// The k-th largest key of each of NR rows held as KPL keys per lane (key j at
-// lane j % 32, slot j / 32; 0 pads, below every real key): the largest T with
-// count(key >= T) >= topk, built most significant bit first.  The NR searches
-// share one bit loop so that their counts and warp reductions overlap.
+// A threshold T for each of NR rows held as KPL keys per lane (key j at lane
+// j % 32, slot j / 32; 0 pads, below every real key) such that the row's topk
+// largest keys are those above T plus the first ones equal to T, in id order:
+// built most significant bit first as the largest T with count(key >= T) >=
+// topk (the k-th largest key), except that a row stops early at the first
+// candidate T with count(key >= T) == topk exactly, whose set {key >= T} is
+// already the row's top-k.  The NR searches share one bit loop, so their
+// counts and warp reductions overlap; a lane counts in four partial sums.
 template <int KPL, int NR>
 __device__ __forceinline__ void kth_largest(const uint32_t (&key)[NR][KPL], int topk, uint32_t (&prefix)[NR]) {
+  bool done[NR];
 #pragma unroll
-  for (int r = 0; r < NR; ++r) prefix[r] = 0u;
+  for (int r = 0; r < NR; ++r) {
+    prefix[r] = 0u;
+    done[r] = false;
+  }
 #pragma unroll 1
   for (int bit = 31; bit >= 0; --bit) {
     uint32_t cnt[NR];
 #pragma unroll
     for (int r = 0; r < NR; ++r) {
       const uint32_t cand = prefix[r] | (1u << bit);
-      uint32_t c = 0;
+      uint32_t c[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-      for (int q = 0; q < KPL; ++q) c += key[r][q] >= cand ? 1u : 0u;
-      cnt[r] = c;
+      for (int q = 0; q < KPL; ++q) c[q & 3] += key[r][q] >= cand ? 1u : 0u;
+      cnt[r] = (c[0] + c[1]) + (c[2] + c[3]);
     }
+    bool all_done = true;
 #pragma unroll
-    for (int r = 0; r < NR; ++r)
-      if (static_cast<int>(__reduce_add_sync(0xffffffffu, cnt[r])) >= topk) prefix[r] |= 1u << bit;
+    for (int r = 0; r < NR; ++r) {
+      const int total = static_cast<int>(__reduce_add_sync(0xffffffffu, cnt[r]));
+      if (!done[r] && total >= topk) {
+        prefix[r] |= 1u << bit;
+        done[r] = total == topk;
+      }
+      all_done = all_done && done[r];
+    }
+    if (all_done) break;   // warp-uniform: the totals are
   }
 }
 
@@ -303,25 +317,28 @@ __global__ void __launch_bounds__(kThreads, 1) score_topk_kernel(const float* __
   score_rows<D, RPW>(qbar, kbar, smem, bh, r0, nrows, nb, a.scores);
   const float* sc = smem + (kRows + kKeys) * (D + 4);
 
-  // top-k: one warp per two rows at a time (r and r + 8 of this warp's share),
-  // the rows' keys in registers
+  // top-k: each warp searches NT rows of its share together (rows r, r + 8, ...,
+  // their keys in registers; NT = 2 for the widest rows, whose keys take 64
+  // registers each); slots past the CTA's last row repeat the pass's first row
+  constexpr int kWarps = kThreads / 32;
+  constexpr int NT = (KPL >= 64 ? 2 : 4) < kRows / kWarps ? (KPL >= 64 ? 2 : 4) : kRows / kWarps;
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int kr = a.head_k == nullptr ? a.topk : min(max(__ldg(a.head_k + bh % a.H), 1), a.topk);
-  for (int r = warp; r < nrows; r += 2 * (kThreads / 32)) {
-    const int r2 = r + kThreads / 32;
-    const bool two = r2 < nrows;
-    const int rr[2] = {r, two ? r2 : r};
-    uint32_t key[2][KPL];
+  for (int r1 = warp; r1 < nrows; r1 += NT * kWarps) {
+    int rr[NT];
+#pragma unroll
+    for (int u = 0; u < NT; ++u) rr[u] = r1 + u * kWarps < nrows ? r1 + u * kWarps : r1;
+    uint32_t key[NT][KPL];
 #pragma unroll
     for (int q = 0; q < KPL; ++q)
 #pragma unroll
-      for (int u = 0; u < 2; ++u) key[u][q] = select_key(sc + rr[u] * nb, q * 32 + lane, r0 + rr[u], a);
-    uint32_t kth[2];
-    kth_largest<KPL, 2>(key, kr, kth);
+      for (int u = 0; u < NT; ++u) key[u][q] = select_key(sc + rr[u] * nb, q * 32 + lane, r0 + rr[u], a);
+    uint32_t kth[NT];
+    kth_largest<KPL, NT>(key, kr, kth);
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      if (u == 1 && !two) break;
+    for (int u = 0; u < NT; ++u) {
+      if (u > 0 && rr[u] == r1) break;
       const size_t row = static_cast<size_t>(bh) * nb + r0 + rr[u];
       compact_row<KPL>(key[u], kth[u], nb, kr, a.idx + row * a.topk, lane);
       finish_row(a, row, kr, lane);
