@@ -42,7 +42,7 @@ def _stale() -> bool:
 
 
 # Kernels whose spilling would silently cost performance: the build refuses them.
-NO_SPILL_KERNELS = ("sparse_attn_fwd_kernel", "sparse_attn_fp8_kernel")
+NO_SPILL_KERNELS = ("sparse_attn_fwd_kernel", "sparse_attn_fp8_kernel", "qk_prologue_pool_staged_kernel")
 # Register ceilings that launches need: a CTA's warps are spread over the SM's four
 # sub-partitions of 16 K registers each, so 10 warps (3 on some sub-partitions) get
 # at most 168 per thread; a kernel built above that fails to launch.

@@ -321,5 +321,204 @@ __global__ void __launch_bounds__(256) qk_prologue_pool_kernel(const Params p, c
   }
 }
 
+// ------------------------------------------------------------------ staged prologue + block pooling
+// bf16, D = 128: the arithmetic of qk_prologue_pool_kernel (same norm_rotate,
+// same per-block summation order, so the same bits), with the data movement
+// organised for HBM.  One persistent CTA per SM walks the (b, block) units
+// blockIdx.x, blockIdx.x + gridDim.x, ...; a producer warp copies each token's
+// whole Q and K rows (all heads: H * 256 contiguous bytes each in [B, N, H, D])
+// into a ring of shared-memory stages with bulk async copies, so that up to
+// `stages` tokens per SM are in flight without holding registers, and writes
+// the token's rotary table offsets beside them.  Sixteen consumer warps (32
+// groups of 16 lanes; group g owns heads g + 32 i, i < HPG) normalise, rotate and
+// store from shared memory, accumulate the block means in registers, and hand
+// each stage back once read.  Every wait is bounded.
+namespace staged {
+constexpr int kConsumerWarps = 16;
+constexpr int kThreads = 32 * (kConsumerWarps + 1);
+constexpr int kGroups = kConsumerWarps * 2;
+constexpr int kMaxStages = 16;
+constexpr int kHeaderBytes = 1024;   // full[16] | empty[16] | meta[16] (int4) | abort flag
+enum : unsigned { kSiteStageFull = 33, kSiteStageFree, kSiteStageTail };
+// Shared-memory offset of the stage ring (after the header and the rotary table).
+__host__ __device__ constexpr int stage_offset(int tab_total) {
+  return (kHeaderBytes + tab_total * 8 + 127) / 128 * 128;
+}
+}  // namespace staged
+
+__device__ __forceinline__ void load_vec_smem(const unsigned char* p, float (&x)[8]) {
+  const uint4 v = *reinterpret_cast<const uint4*>(p);
+  x[0] = __uint_as_float(v.x << 16); x[1] = __uint_as_float(v.x & 0xFFFF0000u);
+  x[2] = __uint_as_float(v.y << 16); x[3] = __uint_as_float(v.y & 0xFFFF0000u);
+  x[4] = __uint_as_float(v.z << 16); x[5] = __uint_as_float(v.z & 0xFFFF0000u);
+  x[6] = __uint_as_float(v.w << 16); x[7] = __uint_as_float(v.w & 0xFFFF0000u);
+}
+
+// grid: min(B * nb, SMs); stages in [2, kMaxStages], each 2 * H * 256 bytes.
+// kPool = false: the plain prologue (no means; qbar, kbar unused), walked in
+// runs of bm.block consecutive tokens.
+template <int HPG, bool kPool>
+__global__ void __launch_bounds__(staged::kThreads, 1)
+    qk_prologue_pool_staged_kernel(const Params p, const BlockMap bm, int nb, int stages, float* qbar, float* kbar) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  constexpr int D = 128, V = 8, L = 16;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem_raw);
+  uint64_t* empty = full + staged::kMaxStages;
+  int4* meta = reinterpret_cast<int4*>(empty + staged::kMaxStages);   // (n, t*pt, y*ph, x*pw) per stage
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(meta + staged::kMaxStages);
+  float2* tab = reinterpret_cast<float2*>(smem_raw + staged::kHeaderBytes);
+  unsigned char* ring = smem_raw + staged::stage_offset(p.tab_total);
+  const uint32_t row_bytes = static_cast<uint32_t>(p.H) * D * 2;
+  const uint32_t stage_bytes = 2 * row_bytes;
+  const int pt = p.dt / 2, ph = p.dh / 2, pw = p.dw / 2;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < stages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], staged::kConsumerWarps);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  for (int i = threadIdx.x; i < p.tab_total; i += blockDim.x) {
+    int pos, pair, d_axis;
+    if (i < p.tab_t) { pos = i / pt; pair = i % pt; d_axis = p.dt; }
+    else if (i < p.tab_h) { pos = (i - p.tab_t) / ph; pair = (i - p.tab_t) % ph; d_axis = p.dh; }
+    else { pos = (i - p.tab_h) / pw; pair = (i - p.tab_h) % pw; d_axis = p.dw; }
+    const double angle = static_cast<double>(pos) * exp2(-p.log2_theta * (2.0 * pair) / d_axis);
+    double sn, cn;
+    sincos(angle, &sn, &cn);
+    tab[i] = make_float2(static_cast<float>(cn), static_cast<float>(sn));
+  }
+  __syncthreads();
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int units = (p.tokens / p.N) * nb;
+  const int hw = p.gh * p.gw;
+  auto unit_tokens = [&](int bi) { return bm.tw == 0 ? min(bm.block, p.N - bi * bm.block) : bm.block; };
+
+  if (warp == staged::kConsumerWarps) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      uint32_t s = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        const int b = u / nb, bi = u - b * nb;
+        const int cnt = unit_tokens(bi);
+        for (int l = 0; l < cnt; ++l, ++s) {
+          const int st = static_cast<int>(s % stages);
+          if (s >= static_cast<uint32_t>(stages) &&
+              !mbar_wait(&empty[st], (s / stages - 1) & 1, abort_flag, staged::kSiteStageFree)) {
+            ok = false;
+            break;
+          }
+          const int n = block_token(bm, bi, l);
+          meta[st] = make_int4(n, (n / hw) * pt, ((n / p.gw) % p.gh) * ph, (n % p.gw) * pw);
+          const size_t off = (static_cast<size_t>(b) * p.N + n) * row_bytes;
+          unsigned char* dst = ring + static_cast<size_t>(st) * stage_bytes;
+          mbar_arrive_expect_tx(&full[st], stage_bytes);
+          bulk_load(dst, static_cast<const unsigned char*>(p.q_in) + off, row_bytes, &full[st]);
+          bulk_load(dst + row_bytes, static_cast<const unsigned char*>(p.k_in) + off, row_bytes, &full[st]);
+        }
+      }
+      // every copy issued completes before the CTA exits (on the abort path too)
+      const uint32_t first = s > static_cast<uint32_t>(stages) ? s - stages : 0u;
+      for (uint32_t i = first; i < s; ++i)
+        mbar_wait(&full[i % stages], (i / stages) & 1, abort_flag, staged::kSiteStageTail, SOL_WAIT_LIMIT_NS, false);
+    }
+    return;
+  }
+
+  // ------------------------------------------------------------------ consumers
+  const int grp = threadIdx.x / L;               // 0 .. kGroups - 1
+  const int lane_in_row = threadIdx.x % L;
+  const unsigned seg = 0xffffu << (lane & 16);
+  float gq[HPG][V], gk[HPG][V];
+#pragma unroll
+  for (int i = 0; i < HPG; ++i) {
+    const int h = min(grp + staged::kGroups * i, p.H - 1);
+#pragma unroll
+    for (int e = 0; e < V; ++e) {
+      gq[i][e] = __ldg(p.gamma_q + h * D + lane_in_row * V + e);
+      gk[i][e] = __ldg(p.gamma_k + h * D + lane_in_row * V + e);
+    }
+  }
+  int axis[V / 2], slot[V / 2];
+#pragma unroll
+  for (int e = 0; e < V / 2; ++e) {
+    const int c = lane_in_row * V + 2 * e;
+    if (c < p.dt) { axis[e] = 0; slot[e] = c / 2; }
+    else if (c < p.dt + p.dh) { axis[e] = 1; slot[e] = p.tab_t + (c - p.dt) / 2; }
+    else { axis[e] = 2; slot[e] = p.tab_h + (c - p.dt - p.dh) / 2; }
+  }
+  __nv_bfloat16* qo = static_cast<__nv_bfloat16*>(p.q_out);
+  __nv_bfloat16* ko = static_cast<__nv_bfloat16*>(p.k_out);
+  uint32_t s = 0;
+  bool ok = true;
+  for (int u = blockIdx.x; u < units; u += gridDim.x) {
+    const int b = u / nb, bi = u - b * nb;
+    const int cnt = unit_tokens(bi);
+    const float inv = 1.0f / static_cast<float>(cnt);
+    float aq[HPG][V], ak[HPG][V];
+#pragma unroll
+    for (int i = 0; i < HPG; ++i)
+#pragma unroll
+      for (int e = 0; e < V; ++e) {
+        aq[i][e] = 0.f;
+        ak[i][e] = 0.f;
+      }
+    for (int l = 0; l < cnt; ++l, ++s) {
+      const int st = static_cast<int>(s % stages);
+      ok = mbar_wait(&full[st], (s / stages) & 1, abort_flag, staged::kSiteStageFull);
+      if (!__all_sync(0xffffffffu, ok)) {
+        ok = false;
+        break;
+      }
+      const int4 m = meta[st];
+      float2 cs[V / 2];
+#pragma unroll
+      for (int e = 0; e < V / 2; ++e) cs[e] = tab[slot[e] + (axis[e] == 0 ? m.y : (axis[e] == 1 ? m.z : m.w))];
+      const unsigned char* src = ring + static_cast<size_t>(st) * stage_bytes + lane_in_row * V * 2;
+      const size_t obase = (static_cast<size_t>(b) * p.N + m.x) * p.H * D + lane_in_row * V;
+#pragma unroll
+      for (int i = 0; i < HPG; ++i) {
+        const int h = grp + staged::kGroups * i;
+        if (h < p.H) {
+          float xq[V], xk[V];
+          load_vec_smem(src + h * D * 2, xq);
+          load_vec_smem(src + row_bytes + h * D * 2, xk);
+          norm_rotate<V, L>(xq, gq[i], cs, seg, D, p.eps);
+          norm_rotate<V, L>(xk, gk[i], cs, seg, D, p.eps);
+          if constexpr (kPool) {
+            store_vec_acc(qo + obase + h * D, xq, aq[i]);
+            store_vec_acc(ko + obase + h * D, xk, ak[i]);
+          } else {
+            store_vec(qo + obase + h * D, xq);
+            store_vec(ko + obase + h * D, xk);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[st]);
+    }
+    if (!ok) break;
+    if constexpr (!kPool) continue;
+#pragma unroll
+    for (int i = 0; i < HPG; ++i) {
+      const int h = grp + staged::kGroups * i;
+      if (h < p.H) {
+        float* dq = qbar + ((static_cast<size_t>(b) * p.H + h) * nb + bi) * D + lane_in_row * V;
+        float* dk = kbar + ((static_cast<size_t>(b) * p.H + h) * nb + bi) * D + lane_in_row * V;
+#pragma unroll
+        for (int e = 0; e < V; e += 4) {
+          *reinterpret_cast<float4*>(dq + e) =
+              make_float4(aq[i][e] * inv, aq[i][e + 1] * inv, aq[i][e + 2] * inv, aq[i][e + 3] * inv);
+          *reinterpret_cast<float4*>(dk + e) =
+              make_float4(ak[i][e] * inv, ak[i][e + 1] * inv, ak[i][e + 2] * inv, ak[i][e + 3] * inv);
+        }
+      }
+    }
+  }
+}
+
 }  // namespace prologue
 }  // namespace sol

@@ -78,6 +78,7 @@ struct DeviceInfo {
   int sm_count = 0;
   unsigned long long ctx_id = 0;   // context the attribute flags below were set in
   bool attn_attr = false, attn_fp8_attr = false;
+  bool prologue_staged_attr[2] = {};   // qk_prologue_pool_staged_kernel without / with block means
   bool select_attr[32] = {};   // score_topk / score_topp_kernel instantiations with the shared-memory opt-in set
 };
 DeviceInfo g_dev[kMaxDevices];
@@ -92,6 +93,7 @@ sol_status device_info(DeviceInfo** out) {
   DeviceInfo& d = g_dev[dev];
   if (ctx == 0 || ctx != d.ctx_id) {   // kernel attributes belong to a context: set them again in this one
     d.attn_attr = d.attn_fp8_attr = false;
+    d.prologue_staged_attr[0] = d.prologue_staged_attr[1] = false;
     for (bool& f : d.select_attr) f = false;
     d.ctx_id = ctx;
   }
@@ -316,6 +318,38 @@ sol_status prologue_params(const void* q_raw, const void* k_raw, void* q_out, vo
   return SOL_OK;
 }
 
+// The staged prologue (bf16, D = 128, H <= 32, the ring fits in shared memory):
+// with block means when qbar_out is given, else plain over runs of 128 tokens.
+// *launched stays false where the shape needs the register-streaming kernels.
+sol_status launch_prologue_staged(const sol::prologue::Params& p, const sol_shape& s, sol_dtype dt,
+                                  const sol::BlockMap& bm, int nb, float* qbar_out, float* kbar_out,
+                                  cudaStream_t stream, bool* launched) {
+  namespace ps = sol::prologue::staged;
+  *launched = false;
+  if (dt != SOL_BF16 || s.D != 128 || s.H > ps::kGroups) return SOL_OK;
+  constexpr int kMaxSmem = 227 * 1024;
+  const int off = ps::stage_offset(p.tab_total);
+  const int stage_bytes = 2 * s.H * 128 * 2;
+  const int stages = std::min(8, (kMaxSmem - off) / stage_bytes);
+  if (stages < 2) return SOL_OK;
+  DeviceInfo* di = nullptr;
+  if (sol_status st = device_info(&di)) return st;
+  const bool pool = qbar_out != nullptr;
+  auto kern = pool ? sol::prologue::qk_prologue_pool_staged_kernel<1, true>
+                   : sol::prologue::qk_prologue_pool_staged_kernel<1, false>;
+  bool& attr = di->prologue_staged_attr[pool ? 1 : 0];
+  if (!attr) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem) != cudaSuccess)
+      return SOL_ERR_CUDA;
+    attr = true;
+  }
+  const size_t total = static_cast<size_t>(off) + static_cast<size_t>(stages) * stage_bytes;
+  const int units = s.B * nb;
+  kern<<<std::min(units, di->sm_count), ps::kThreads, total, stream>>>(p, bm, nb, stages, qbar_out, kbar_out);
+  *launched = true;
+  return SOL_OK;
+}
+
 // The fused prologue + block means for any block map.
 sol_status prologue_pool_impl(const void* q_raw, const void* k_raw, void* q_out, void* k_out, const float* gamma_q,
                               const float* gamma_k, sol_shape s, int rope_dt, int rope_dh, int rope_dw,
@@ -331,6 +365,9 @@ sol_status prologue_pool_impl(const void* q_raw, const void* k_raw, void* q_out,
   const int nb = blocks_of(s, bm);
   if (nb > 65535 || s.B > 65535) return SOL_ERR_UNSUPPORTED;
   const dim3 grid(nb, s.B);
+  bool launched = false;
+  if (sol_status st = launch_prologue_staged(p, s, dt, bm, nb, qbar_out, kbar_out, stream, &launched)) return st;
+  if (launched) return launch_status();
   if (dt == SOL_BF16) {
     if (s.D == 128)
       sol::prologue::qk_prologue_pool_kernel<__nv_bfloat16, 128><<<grid, 256, smem, stream>>>(p, bm, nb, qbar_out,
@@ -377,6 +414,13 @@ sol_status sol_qk_prologue(const void* q_raw, const void* k_raw, void* q_out, vo
   if (sol_status st = prologue_params(q_raw, k_raw, q_out, k_out, gamma_q, gamma_k, s, rope_dt, rope_dh, rope_dw,
                                       rope_theta, eps, dt, &p, &smem))
     return st;
+  {
+    const sol::BlockMap runs = sol::raster_blocks(128, s.grid_h, s.grid_w);
+    bool launched = false;
+    if (sol_status st = launch_prologue_staged(p, s, dt, runs, (s.N + 127) / 128, nullptr, nullptr, stream, &launched))
+      return st;
+    if (launched) return launch_status();
+  }
   DeviceInfo* di = nullptr;
   if (sol_status st = device_info(&di)) return st;
   // Every row group keeps one head: the number of groups must be a multiple of H.

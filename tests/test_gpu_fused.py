@@ -11,7 +11,8 @@ sol_block_select_pooled.
     id (both pool in ascending token order in fp32), and so passes the same
     oracle selection rule.
 Covered: the fp32 workload (4x16x16 grid, block 64, k = 4 and 16), a small bf16
-case with a ragged last block, and the 896x512 workload at full size.
+case with a ragged last block, a small bf16 case with 40 heads, and the 896x512
+workload at full size.
 """
 import numpy as np
 import pytest
@@ -74,6 +75,14 @@ def test_fused_small_bf16_ragged_block(sol):
                   grid=(3, 8, 40), block=128, topk=(3,))
     assert wl.N % wl.block == 64
     run_case(sol, wl, make_inputs(wl, seed=5), (1, 3, wl.nb))
+
+
+def test_fused_small_bf16_many_heads(sol):
+    # 40 heads: more than the staged kernel's 32 row groups, so both prologue
+    # entry points take the register-streaming kernels
+    wl = Workload(config_id=91, name="small bf16, 40 heads", dtype="bf16", B=1, H=40, D=128,
+                  grid=(2, 8, 24), block=128, topk=(2,))
+    run_case(sol, wl, make_inputs(wl, seed=6), (1, 2, wl.nb))
 
 
 def test_fused_workload1_bf16_full(sol):

@@ -21,8 +21,11 @@ def rand(shape, dtype, seed, scale=1.0, offset=None):
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
-@pytest.mark.parametrize("D,grid,H,B", [(128, (3, 5, 7), 3, 2), (64, (2, 9, 11), 4, 1), (128, (1, 1, 50), 1, 1)])
+@pytest.mark.parametrize("D,grid,H,B", [(128, (3, 5, 7), 3, 2), (64, (2, 9, 11), 4, 1), (128, (1, 1, 50), 1, 1),
+                                        (128, (2, 3, 5), 40, 1)])
 def test_prologue_small(sol, dtype, D, grid, H, B):
+    # bf16 with D = 128 runs the shared-memory staged kernel up to 32 heads and the
+    # register-streaming one above (H = 40)
     N = grid[0] * grid[1] * grid[2]
     q_raw, k_raw = rand((B, N, H, D), dtype, 1), rand((B, N, H, D), dtype, 2, 2.0)
     gq = torch.rand(H * D, generator=torch.Generator().manual_seed(3)) * 0.4 + 0.8
