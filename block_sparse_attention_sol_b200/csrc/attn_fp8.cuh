@@ -274,6 +274,31 @@ sparse_attn_fp8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
     const uint32_t lanes16 = static_cast<uint32_t>(quad * 32 + half * 16) << 16;
     const uint32_t lanes32 = static_cast<uint32_t>(quad * 32) << 16;
     const int tail_valid = p.N - (p.nb - 1) * kBlock;
+    // This thread's 64 Q codes (one row of its quadrant) of tile tt.
+    auto load_q_rows = [&](int tt, uint32_t (&qv)[16]) {
+      int tb, th, tq;
+      decode_tile(p, tt, tb, th, tq);
+      const int nq = tq * kBlock + quad * 32 + lane;
+      if (nq < p.N) {
+        const uint4* src = reinterpret_cast<const uint4*>(
+            p.q + ((static_cast<size_t>(tb) * p.N + nq) * p.H + th) * kHeadDim + 64 * half);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const uint4 w = __ldg(src + c);
+          qv[4 * c] = w.x; qv[4 * c + 1] = w.y; qv[4 * c + 2] = w.z; qv[4 * c + 3] = w.w;
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 16; ++c) qv[c] = 0u;
+      }
+    };
+    auto store_q = [&](const uint32_t (&qv)[16]) {
+      tmem_st32x16(tmem + lanes32 + kColQ + 16 * half, qv);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.q_full);
+    };
     uint32_t g = 0, sq = 0;
     int it = 0;
     bool ok = true;
@@ -283,33 +308,14 @@ sparse_attn_fp8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
       const int32_t* list = p.idx + (static_cast<size_t>(b * p.H + h) * p.nb + qb) * p.topk;
       const float* ksc = p.k_scale + static_cast<size_t>(b * p.H + h) * p.nb;
       const int kt = tile_steps(p, t);
-      if (it > 0) {
-        ok = mbar_wait(&sm.q_empty, (it - 1) & 1, abort_flag, kSiteQEmpty);
-        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-        tc_fence_after();
-      }
-      {
-        // Qc rows into TMEM: lane = row, 4 codes per column; the two warps of a
-        // quadrant write channels [64 half, 64 half + 64) = 16 columns each.
-        const int nq = qb * kBlock + quad * 32 + lane;
+      // Qc rows into TMEM: lane = row, 4 codes per column; the two warps of a quadrant
+      // write channels [64 half, 64 half + 64) = 16 columns each.  The first tile's
+      // Q is stored here; each later tile's Q is loaded during the previous tile's
+      // epilogue, so that its first S products overlap that epilogue.
+      if (it == 0) {
         uint32_t qv[16];
-        if (nq < p.N) {
-          const uint4* src = reinterpret_cast<const uint4*>(
-              p.q + ((static_cast<size_t>(b) * p.N + nq) * p.H + h) * kHeadDim + 64 * half);
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const uint4 w = __ldg(src + c);
-            qv[4 * c] = w.x; qv[4 * c + 1] = w.y; qv[4 * c + 2] = w.z; qv[4 * c + 3] = w.w;
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < 16; ++c) qv[c] = 0u;
-        }
-        tmem_st32x16(tmem + lanes32 + kColQ + 16 * half, qv);
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.q_full);
+        load_q_rows(t, qv);
+        store_q(qv);
       }
       // per-row factor scale * log2(e) * sq[row]
       float rf0 = 0.f, rf1 = 0.f;
@@ -430,6 +436,10 @@ sparse_attn_fp8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
         if (lane == 0) mbar_arrive(&sm.p_full);
       }
       if (!ok) break;
+      // The next tile's Q: loads issued now, stored once this tile's O has been read.
+      const int t_next = t + gridDim.x;
+      uint32_t qn[16];
+      if (t_next < p.num_tiles) load_q_rows(t_next, qn);
       ok = mbar_wait(&sm.pv_done, (g + kt - 1) & 1, abort_flag, kSitePvDone);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
@@ -457,6 +467,12 @@ sparse_attn_fp8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.o_free);
+      if (t_next < p.num_tiles) {
+        ok = mbar_wait(&sm.q_empty, it & 1, abort_flag, kSiteQEmpty);   // this tile's S MMAs done
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        tc_fence_after();
+        store_q(qn);
+      }
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
         const int n = qb * kBlock + row0 + 8 * u;

@@ -260,6 +260,31 @@ sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
     const uint32_t lanes32 = static_cast<uint32_t>(quad * 32) << 16;
     const int tail_valid = p.N - (p.nb - 1) * kBlock;   // valid keys in the last block
     const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
+    // This thread's 64 Q channels (one row of its quadrant) of tile tt, as bf16 pairs.
+    auto load_q_rows = [&](int tt, uint32_t (&qv)[32]) {
+      int tb, th, tq;
+      decode_tile(p, tt, tb, th, tq);
+      const int nq = block_token(p.bm, tq, quad * 32 + lane);
+      if (nq < p.N) {
+        const uint4* src = reinterpret_cast<const uint4*>(
+            p.q + ((static_cast<size_t>(tb) * p.N + nq) * p.H + th) * kHeadDim + 64 * half);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint4 w = __ldg(src + c);
+          qv[4 * c] = w.x; qv[4 * c + 1] = w.y; qv[4 * c + 2] = w.z; qv[4 * c + 3] = w.w;
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) qv[c] = 0u;
+      }
+    };
+    auto store_q = [&](const uint32_t (&qv)[32]) {
+      tmem_st32(tmem + lanes32 + kColQ + 32 * half, qv);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.q_full);
+    };
     uint32_t g = 0;    // steps before this tile
     uint32_t sq = 0;   // K/V slots before this tile (topk + 2 per tile)
     int it = 0;
@@ -270,32 +295,13 @@ sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
       const int32_t* list = p.idx + (static_cast<size_t>(b * p.H + h) * p.nb + qb) * p.topk;
       const int kt = tile_steps(p, t);
       // ---- Q into TMEM (A operand of the S MMAs: lane = row, 2 bf16 per column).
-      // The two warps of a quadrant write channels [64 half, 64 half + 64) of its 32 rows.
-      if (it > 0) {
-        ok = mbar_wait(&sm.q_empty, (it - 1) & 1, abort_flag, kSiteQEmpty);   // previous tile's S MMAs done
-        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-        tc_fence_after();
-      }
-      {
-        const int nq = block_token(p.bm, qb, quad * 32 + lane);
+      // The two warps of a quadrant write channels [64 half, 64 half + 64) of its 32
+      // rows.  The first tile's Q is stored here; each later tile's Q is loaded during
+      // the previous tile's epilogue, so that its first S products overlap that epilogue.
+      if (it == 0) {
         uint32_t qv[32];
-        if (nq < p.N) {
-          const uint4* src = reinterpret_cast<const uint4*>(
-              p.q + ((static_cast<size_t>(b) * p.N + nq) * p.H + h) * kHeadDim + 64 * half);
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const uint4 w = __ldg(src + c);
-            qv[4 * c] = w.x; qv[4 * c + 1] = w.y; qv[4 * c + 2] = w.z; qv[4 * c + 3] = w.w;
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < 32; ++c) qv[c] = 0u;
-        }
-        tmem_st32(tmem + lanes32 + kColQ + 32 * half, qv);
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.q_full);
+        load_q_rows(t, qv);
+        store_q(qv);
       }
       float m0 = -INFINITY, m1 = -INFINITY;   // running max per row, log2 units (stale by < 2^8)
       float l0 = 0.f, l1 = 0.f;               // this thread's part of the running sums
@@ -407,6 +413,12 @@ sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
         blk = blk_next;
       }
       if (!ok) break;
+      // The next tile's Q: global loads issued now, stored into TMEM once this
+      // tile's O has been read below (its S products are complete by then: every
+      // S of this tile has been consumed).
+      const int t_next = t + gridDim.x;
+      uint32_t qn[32];
+      if (t_next < p.num_tiles) load_q_rows(t_next, qn);
       // epilogue: O / l and LSE
       {
         ok = mbar_wait(&sm.pv_done, (g + kt - 1) & 1, abort_flag, kSitePvDone);
@@ -436,6 +448,12 @@ sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_co
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.o_free);
+      if (t_next < p.num_tiles) {
+        ok = mbar_wait(&sm.q_empty, it & 1, abort_flag, kSiteQEmpty);   // this tile's S MMAs done
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        tc_fence_after();
+        store_q(qn);
+      }
       // The four threads of a row hold its channel pairs 8i + 2c (thread c); a 4 x 4
       // exchange per group of four i gives thread c the 16 contiguous bytes of
       // channels 8 (4a + c) .. + 7, which it stores in one instruction.
