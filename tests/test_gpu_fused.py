@@ -118,3 +118,27 @@ def test_host_pipeline_matches_direct_calls(sol):
         assert torch.equal(o.cpu().view(torch.int16), o_host.view(torch.int16))
         assert torch.equal(lse.cpu(), lse_host)
     assert sol.sol_check_device_status() == sol.SOL_OK
+
+
+def test_chain_graph_matches_direct_calls(sol):
+    """The fused chain captured once as a CUDA graph (ChainGraph) and replayed on
+    three clips gives exactly the outputs of the direct calls on each clip."""
+    from block_sparse_attention_sol_b200.graph import ChainGraph
+    wl = Workload(config_id=93, name="graph check, ragged last block", dtype="bf16", B=1, H=4, D=128,
+                  grid=(3, 8, 40), block=128, topk=(3,))
+    topk = 3
+    clips = [make_inputs(wl, seed=s) for s in range(3)]
+    gq, gk = clips[0]["gamma_q"].cuda(), clips[0]["gamma_k"].cuda()
+    chain = ChainGraph(wl.B, wl.N, wl.H, wl.D, wl.grid, wl.block, topk, gq, gk, rope_split=wl.rope_split,
+                       rope_theta=wl.rope_theta, eps=wl.eps).capture()
+    for c in clips:
+        o_g, lse_g = chain(c["q"].cuda(), c["k"].cuda(), c["v"].cuda())
+        o_g, lse_g = o_g.clone(), lse_g.clone()
+        q, k, qbar, kbar = sol.sol_qk_prologue_pool(c["q"].cuda(), c["k"].cuda(), gq, gk, wl.grid, wl.block,
+                                                    wl.rope_split, wl.rope_theta, wl.eps)
+        idx = sol.sol_block_select_pooled(qbar, kbar, wl.grid, wl.block, topk)
+        o, lse = sol.sol_sparse_attn_fwd(q, k, c["v"].cuda(), idx, wl.grid, wl.block)
+        torch.cuda.synchronize()
+        assert torch.equal(o_g.view(torch.int16), o.view(torch.int16))
+        assert torch.equal(lse_g, lse)
+    assert sol.sol_check_device_status() == sol.SOL_OK
