@@ -309,3 +309,19 @@ def test_backward_argument_checks(lib):
     assert call(dq=MISALIGNED) == INVALID
     assert call(dt=5) == INVALID
     assert call(shape=Shape(1, 1024, 2, 96, 4, 16, 16), ws_bytes=1 << 20) == UNSUPPORTED
+
+
+def test_noalloc_select_shape_checks(lib):
+    """The allocation-free selection rejects a malformed shape and one whose pooled
+    means exceed its fixed 40 MiB scratch before touching the device."""
+    f = lib.sol_block_select_noalloc
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p, ctypes.c_void_p, Shape, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                  ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+    wsb = lib.sol_block_select_workspace_bytes
+    wsb.restype = ctypes.c_size_t
+    wsb.argtypes = [Shape, ctypes.c_int]
+    assert f(FAKE, FAKE, Shape(1, 1000, 2, 64, 4, 16, 16), 64, 4, 0, FAKE, None, None) == INVALID  # N != grid
+    big = Shape(1, 16 * 68 * 120, 64, 128, 16, 68, 120)   # 64 heads at 130,560 tokens: 66.8 MB of means
+    assert wsb(big, 128) > 40 * 1024 * 1024
+    assert f(FAKE, FAKE, big, 128, 102, 0, FAKE, None, None) == UNSUPPORTED
