@@ -53,3 +53,22 @@ def test_local_transport_copies():
     dst = torch.zeros(12)
     LocalTransport().all_to_all(dst, src)
     assert torch.equal(dst, src)
+
+
+def test_runners_require_gains_on_their_device():
+    """HostChainPipeline and ChainGraph check, before allocating anything, that the
+    gains live on the device they run on."""
+    from block_sparse_attention_sol_b200.graph import ChainGraph
+    from block_sparse_attention_sol_b200.pipeline import HostChainPipeline
+    gq = gk = torch.ones(2 * 128)
+    for runner in (HostChainPipeline, ChainGraph):
+        with pytest.raises(ValueError, match="device"):
+            runner(1, 1024, 2, 128, (4, 16, 16), 128, 2, gq, gk, device="cuda:0")
+
+
+def test_chain_graph_replay_needs_capture():
+    from block_sparse_attention_sol_b200.graph import ChainGraph
+    g = ChainGraph.__new__(ChainGraph)
+    g.graph = None
+    with pytest.raises(RuntimeError, match="capture"):
+        g.replay()
